@@ -1,0 +1,154 @@
+"""Seeded synthetic inputs for the LSA decode workloads.
+
+Both the CUDA path and the CPU oracle are fed from here; this module holds no
+arithmetic of the method (no projection, scoring, selection or attention), only
+random draws and their bf16 casts (round to nearest even, torch's fp32 -> bf16 copy).
+
+Every tensor is drawn from its own named stream (a torch CPU generator seeded by a
+hash of the workload seed and the stream's name), so any piece -- one pass's hidden
+states, one step's queries, one chunk of the cold pool -- can be regenerated alone,
+and the draws do not depend on the device or the number of threads used.
+
+Distributions (all i.i.d.): W_q ~ N(0, 1/D); h, K_idx, K, V, q ~ N(0, 1); all cast
+to bf16. The KV history of a sequence is drawn for its final context (pass-0
+context plus 64 tokens per pass), so the token decode step s of pass p appends is
+simply history position N_p + s.
+"""
+from __future__ import annotations
+
+import hashlib
+import os
+from concurrent.futures import ThreadPoolExecutor
+from typing import Optional
+
+import numpy as np
+import torch
+
+from .configs import LsaConfig
+
+POOL_CHUNK_BLOCKS = 256
+
+
+def stream_seed(base: int, *keys) -> int:
+    h = hashlib.blake2b(repr((int(base),) + tuple(keys)).encode(), digest_size=8)
+    return int.from_bytes(h.digest(), "little") & ((1 << 63) - 1)
+
+
+def _gen(base: int, *keys) -> torch.Generator:
+    return torch.Generator().manual_seed(stream_seed(base, *keys))
+
+
+def _randn_bf16(shape, gen: torch.Generator, std: float = 1.0) -> torch.Tensor:
+    x = torch.randn(shape, generator=gen, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.bfloat16)
+
+
+class Workload:
+    """All inputs of one LSA decode run (one config)."""
+
+    def __init__(self, cfg: LsaConfig, pin: bool = False, threads: Optional[int] = None):
+        self.cfg = cfg
+        B, blk = cfg.B, cfg.block
+        # context lengths (tokens at pass 0) and per-sequence bias
+        if cfg.ctx_tokens is not None:
+            ctx = np.asarray(cfg.ctx_tokens, dtype=np.int64)
+        else:
+            lo, hi = cfg.ctx_uniform_blocks
+            g = _gen(cfg.seed, "ctx_blocks")
+            ctx = torch.randint(lo, hi + 1, (B,), generator=g).numpy().astype(np.int64) * blk
+        assert ctx.shape == (B,) and np.all(ctx % blk == 0) and np.all(ctx > 0)
+        if cfg.bias is not None:
+            bias = np.asarray(cfg.bias, dtype=np.float32)
+        else:
+            lo, hi = cfg.bias_uniform
+            g = _gen(cfg.seed, "bias")
+            bias = (lo + (hi - lo) * torch.rand((B,), generator=g, dtype=torch.float64)).numpy()
+            bias = bias.astype(np.float32)
+        self.ctx0 = ctx
+        self.nb0 = ctx // blk
+        self.nb_final = self.nb0 + cfg.passes
+        self.bias = bias
+        off = np.zeros(B + 1, dtype=np.int64)
+        off[1:] = np.cumsum(self.nb_final)
+        self.blk_off = off            # first block of sequence b in k_idx and in the host pool
+        self.total_blocks = int(off[-1])
+
+        self.w_q = _randn_bf16((cfg.L, cfg.d_i, cfg.D), _gen(cfg.seed, "w_q"), cfg.wq_std)
+        self.k_idx = torch.empty((self.total_blocks, cfg.d_i), dtype=torch.bfloat16)
+        for b in range(B):
+            self.k_idx[off[b]:off[b + 1]] = _randn_bf16(
+                (int(self.nb_final[b]), cfg.d_i), _gen(cfg.seed, "k_idx", b))
+        self.host_pool = torch.empty((self.total_blocks, 2, blk, cfg.d), dtype=torch.bfloat16,
+                                     pin_memory=pin)
+        self._fill_pool(threads)
+
+    # -- cold pool ---------------------------------------------------------------
+    def _fill_pool(self, threads):
+        n = self.total_blocks
+        flat = self.host_pool.view(n, -1)
+        chunks = [(i, min(i + POOL_CHUNK_BLOCKS, n)) for i in range(0, n, POOL_CHUNK_BLOCKS)]
+        seed = self.cfg.seed
+
+        def work(c):
+            lo, hi = c
+            x = torch.randn((hi - lo, flat.shape[1]), generator=_gen(seed, "pool", lo),
+                            dtype=torch.float32)
+            flat[lo:hi].copy_(x)
+
+        nthr = threads or min(32, os.cpu_count() or 1)
+        if len(chunks) == 1 or nthr == 1:
+            for c in chunks:
+                work(c)
+            return
+        old = torch.get_num_threads()
+        torch.set_num_threads(1)
+        try:
+            with ThreadPoolExecutor(nthr) as ex:
+                list(ex.map(work, chunks))
+        finally:
+            torch.set_num_threads(old)
+
+    # -- per pass / per step draws -------------------------------------------------
+    def ctx_at(self, p: int) -> np.ndarray:
+        """Tokens of each sequence's context when pass p starts."""
+        return self.ctx0 + self.cfg.tau * p
+
+    def h(self, p: int) -> torch.Tensor:
+        """Hidden states the indexer reads at the start of pass p: bf16 [L][B][D]."""
+        c = self.cfg
+        return _randn_bf16((c.L, c.B, c.D), _gen(c.seed, "h", p))
+
+    def q(self, p: int, s: int) -> torch.Tensor:
+        """Queries of decode step s of pass p: bf16 [B][H][d]."""
+        c = self.cfg
+        return _randn_bf16((c.B, c.H, c.d), _gen(c.seed, "q", p, s))
+
+    def token_kv(self, b: int, pos: int):
+        """(K, V) bf16 [d] of history position pos of sequence b."""
+        blk = self.cfg.block
+        page = self.host_pool[self.blk_off[b] + pos // blk]
+        return page[0, pos % blk], page[1, pos % blk]
+
+    def kv_new(self, p: int, s: int):
+        """The token appended at step s of pass p: (k, v) bf16 [B][d] each."""
+        pos = self.ctx_at(p) + s
+        ks = torch.stack([self.token_kv(b, int(pos[b]))[0] for b in range(self.cfg.B)])
+        vs = torch.stack([self.token_kv(b, int(pos[b]))[1] for b in range(self.cfg.B)])
+        return ks, vs
+
+    def seq_kv(self, b: int):
+        """Views K, V bf16 [tokens][d] over the whole drawn history of sequence b."""
+        pages = self.host_pool[self.blk_off[b]:self.blk_off[b + 1]]
+        d = self.cfg.d
+        return pages[:, 0].reshape(-1, d), pages[:, 1].reshape(-1, d)
+
+    def seq_k_idx(self, b: int) -> torch.Tensor:
+        return self.k_idx[self.blk_off[b]:self.blk_off[b + 1]]
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """The raw bf16 bit patterns of a tensor, as a numpy uint16 array (no conversion)."""
+    assert t.dtype == torch.bfloat16
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
