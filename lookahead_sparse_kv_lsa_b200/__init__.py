@@ -1,0 +1,127 @@
+"""Lookahead Sparse Attention (LSA) decode hot path for B200 (sm_100a).
+
+Thin Python binding over the C ABI of include/lsa.h: every function below only checks
+and marshals torch tensors (device memory, streams) into the library's entry points.
+All computation happens in the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import LsaError, LsaState, BLOCK, TAU
+
+__all__ = ["lsa_index", "lsa_gather", "lsa_decode_attn", "lsa_step", "lsa_load_window",
+           "index_workspace_size", "decode_attn_workspace_size", "LsaDecoder", "LsaError",
+           "LsaState", "BLOCK", "TAU", "library_path"]
+
+
+def library_path() -> str:
+    return _lib.LIB_PATH
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str, numel: Optional[int] = None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if numel is not None and t.numel() < numel:
+        raise ValueError("%s holds %d elements, needs %d" % (name, t.numel(), numel))
+    return t.data_ptr()
+
+
+def _opt(t, dtype, name, numel=None) -> Optional[int]:
+    return None if t is None else _dev(t, dtype, name, numel)
+
+
+def index_workspace_size(B: int, L: int, d_i: int, max_cand: int) -> int:
+    return int(_lib.lib().lsa_index_workspace_size(B, L, d_i, max_cand))
+
+
+def decode_attn_workspace_size(B: int, H: int, d: int, n_sm: Optional[int] = None) -> int:
+    if n_sm is None:
+        n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return int(_lib.lib().lsa_decode_attn_workspace_size(B, H, d, n_sm))
+
+
+def lsa_index(h, w_q, bias, k_idx, kidx_off, n_cand, max_cand: int, sel_ids, sel_cnt, ws, err,
+              logits=None, layer_mask=None, stream=None) -> None:
+    """One indexer pass; see lsa_index in include/lsa.h. h [L][B][D], w_q [L][d_i][D]."""
+    L, B, D = h.shape
+    d_i = w_q.shape[1]
+    cap = sel_ids.shape[1] if sel_ids.dim() == 2 else 0
+    st = _lib.lib().lsa_index(
+        _dev(h, torch.bfloat16, "h"), _dev(w_q, torch.bfloat16, "w_q", L * d_i * D),
+        _dev(bias, torch.float32, "bias", B), _dev(k_idx, torch.bfloat16, "k_idx"),
+        _dev(kidx_off, torch.int64, "kidx_off", B), _dev(n_cand, torch.int32, "n_cand", B),
+        B, L, D, d_i, max_cand,
+        _dev(sel_ids, torch.int32, "sel_ids"), _dev(sel_cnt, torch.int32, "sel_cnt", B), cap,
+        _opt(logits, torch.float32, "logits", L * B * max_cand),
+        _opt(layer_mask, torch.int32, "layer_mask", (L + 1) * B * ((max_cand + 31) // 32)),
+        _dev(ws, torch.uint8, "ws"), ws.numel(), _dev(err, torch.int32, "err", 1), _stream(stream))
+    _lib.check("lsa_index", st)
+
+
+def lsa_gather(host_pool, host_blk_off, sel_ids, sel_cnt, res_pages, n_res, hbm_pool,
+               sel_page_base: int, sel_page_count: int, block_table, n_entries, err,
+               stream=None) -> None:
+    """Copy kept blocks host pool -> HBM pool and build block tables (lsa_gather in lsa.h)."""
+    if host_pool.is_cuda or not host_pool.is_pinned() or host_pool.dtype != torch.bfloat16:
+        raise ValueError("host_pool must be a pinned host bf16 tensor")
+    B = sel_cnt.shape[0]
+    d = hbm_pool.shape[-1]
+    st = _lib.lib().lsa_gather(
+        host_pool.data_ptr(), host_pool.shape[0], _dev(host_blk_off, torch.int64, "host_blk_off", B),
+        _dev(sel_ids, torch.int32, "sel_ids"), _dev(sel_cnt, torch.int32, "sel_cnt", B),
+        sel_ids.shape[1], _dev(res_pages, torch.int32, "res_pages"),
+        _dev(n_res, torch.int32, "n_res", B), res_pages.shape[1], B, d,
+        _dev(hbm_pool, torch.bfloat16, "hbm_pool"), hbm_pool.shape[0], sel_page_base,
+        sel_page_count, _dev(block_table, torch.int32, "block_table"), block_table.shape[1],
+        _dev(n_entries, torch.int32, "n_entries", B), _dev(err, torch.int32, "err", 1),
+        _stream(stream))
+    _lib.check("lsa_gather", st)
+
+
+def lsa_decode_attn(q, hbm_pool, block_table, n_entries, tail_len, scale: float, out, ws, err,
+                    stream=None) -> None:
+    """One block-sparse MQA decode step (lsa_decode_attn in lsa.h). q, out: [B][H][d] bf16."""
+    B, H, d = q.shape
+    st = _lib.lib().lsa_decode_attn(
+        _dev(q, torch.bfloat16, "q"), _dev(hbm_pool, torch.bfloat16, "hbm_pool"),
+        hbm_pool.shape[0], _dev(block_table, torch.int32, "block_table"), block_table.shape[1],
+        _dev(n_entries, torch.int32, "n_entries", B), _dev(tail_len, torch.int32, "tail_len", B),
+        B, H, d, float(scale), _dev(out, torch.bfloat16, "out", B * H * d),
+        _dev(ws, torch.uint8, "ws"), ws.numel(), _dev(err, torch.int32, "err", 1),
+        _stream(stream))
+    _lib.check("lsa_decode_attn", st)
+
+
+def lsa_load_window(state: LsaState, pass_idx: int, stream=None) -> None:
+    _lib.check("lsa_load_window", _lib.lib().lsa_load_window(C.byref(state), pass_idx,
+                                                               _stream(stream)))
+
+
+def lsa_step(state: LsaState, step: int, h, q, k_new, v_new, out, stream=None) -> None:
+    """One decode step of the LSA loop (lsa_step in lsa.h)."""
+    hp = None if h is None else _dev(h, torch.bfloat16, "h")
+    st = _lib.lib().lsa_step(C.byref(state), step, hp, _dev(q, torch.bfloat16, "q"),
+                             _dev(k_new, torch.bfloat16, "k_new"),
+                             _dev(v_new, torch.bfloat16, "v_new"),
+                             _dev(out, torch.bfloat16, "out"), _stream(stream))
+    _lib.check("lsa_step", st)
+
+
+from .decoder import LsaDecoder  # noqa: E402

@@ -1,0 +1,753 @@
+// Block-sparse split-K flash-decode MQA attention on the sm_100a tensor cores, and the
+// log-sum-exp merge of its partial results.
+//
+// One decode step of section 2, step 4 of "FlashMemory-DeepSeek-V4 Explained"
+// (zhichai.net): the query heads of a sequence attend only to the KV pages listed in its
+// block table (the kept blocks, the recent window, the tail page of new tokens).
+//
+// Work split. A sequence's tokens are cut into 32-token units (a page is two units; the
+// tail page ceil(tail_len/32)). All units of the batch, in sequence order, are divided
+// evenly over the grid (one CTA per SM), so a CTA may finish one sequence and start the
+// next; each (CTA, sequence) piece is a "segment" that leaves one partial result
+// (unnormalised O, running max m, sum l) in the workspace slot CTA + sequence. Within a
+// segment, tiles of 128 tokens (4 units) are processed in a software pipeline:
+//
+//   warp 0  TMA producer: Q once per segment, then K and V of each tile, in 16 KB
+//           stages of [128 tokens][64 dims] (128-byte swizzle) through an 8-stage ring;
+//   warp 1  MMA issuer (one thread): S^T[tok][head] = K . Q^T into tensor memory
+//           (M = 128 tokens, N = heads, K = d), then O^T[dim][head] += V^T . P^T
+//           (M = 128 dims per MMA, N = heads, K = 128 tokens), accumulated in TMEM;
+//   warps 2-5 softmax: each owns 32 rows (tokens) of S^T, finds the per-head tile max
+//           (warp butterfly + shared memory), keeps a running max per head that is only
+//           raised when the tile max exceeds it by more than 2^8 (O^T in TMEM is then
+//           rescaled), writes P^T = exp2(S*scale*log2e - m) as bf16 into shared memory,
+//           and accumulates the per-head denominators in registers.
+//
+// Tensor memory columns: S^T double buffer [0, 2*HP), O^T blocks [2*HP, 2*HP + HP*d/128).
+#include "lsa_common.cuh"
+
+#include <math.h>
+
+namespace lsa {
+namespace attn {
+
+constexpr int TILE = 128;                 // tokens per tile (the MMA M of S^T)
+constexpr int UNIT = 32;                  // tokens per work unit (rows per TMA box)
+constexpr int NST = 8;                    // stages in the K/V ring (even: V pairs stay adjacent)
+constexpr int STAGE_BYTES = TILE * 128;   // [128 rows][64 bf16] = 16 KB
+constexpr int NTHREADS = 192;
+constexpr int MAXSEG = 16;                // segments planned per batch
+constexpr float RESCALE_LOG2 = 8.0f;      // raise the running max only by more than 2^8
+
+struct Seg {
+  int b, u0, u1;
+};
+
+struct Misc {
+  uint64_t full[NST], empty[NST];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, pv_done, q_full, q_free, mma_done;
+  uint32_t tmem_base;
+  int abort;
+  int nseg, more;
+  Seg seg[MAXSEG];
+  float red[4][64];
+  float m_use[64];
+  float alpha[64];
+};
+
+struct Args {
+  const int32_t* block_table;
+  const int32_t* n_entries;
+  const int32_t* tail_len;
+  float* part_o;    // [slots][H][d] fp32
+  float* part_ml;   // [slots][H][2] fp32 (running max in log2 units, denominator)
+  int32_t* err;
+  long long n_pages;
+  int bt_stride, B, H, d;
+  float scale_log2;
+};
+
+// Units (32-token pieces) of sequence b; 0 for an empty or malformed sequence.
+__device__ __forceinline__ int seq_units(const Args& a, int b) {
+  const int n = __ldg(a.n_entries + b);
+  if (n <= 0) return 0;
+  const int t = __ldg(a.tail_len + b);
+  if (n > a.bt_stride || t < 1 || t > 64) return 0;
+  return 2 * (n - 1) + (t + UNIT - 1) / UNIT;
+}
+
+__device__ __forceinline__ bool seq_malformed(const Args& a, int b) {
+  const int n = __ldg(a.n_entries + b);
+  if (n < 0) return true;
+  if (n == 0) return false;
+  const int t = __ldg(a.tail_len + b);
+  return n > a.bt_stride || t < 1 || t > 64;
+}
+
+// Total units of the batch, summed by one warp (all lanes get the result).
+__device__ __forceinline__ long long warp_total_units(const Args& a, int lane) {
+  long long s = 0;
+  for (int b = lane; b < a.B; b += 32) s += seq_units(a, b);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+// Warp 0: list the segments of units [us, ue), skipping the first `skip` of them; at most
+// MAXSEG are stored. Sets m->more when segments remain after the stored ones.
+__device__ void plan_segments(const Args& a, long long us, long long ue, int skip, Misc* m,
+                              int lane) {
+  int found = 0, stored = 0;
+  bool more = false;
+  long long base = 0;
+  for (int b0 = 0; b0 < a.B && base < ue && !more; b0 += 32) {
+    const int b = b0 + lane;
+    const int u = b < a.B ? seq_units(a, b) : 0;
+    long long incl = u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const long long p = base + incl - u;  // first unit of sequence b
+    const bool hit = u > 0 && us < ue && p < ue && p + u > us;
+    const unsigned mask = __ballot_sync(0xffffffffu, hit);
+    if (hit) {
+      const int idx = found + __popc(mask & ((1u << lane) - 1u)) - skip;
+      if (idx >= MAXSEG) {
+        more = true;
+      } else if (idx >= 0) {
+        Seg s;
+        s.b = b;
+        s.u0 = static_cast<int>(us > p ? us - p : 0);
+        s.u1 = static_cast<int>((ue < p + u ? ue : p + u) - p);
+        m->seg[idx] = s;
+      }
+    }
+    more = __any_sync(0xffffffffu, more);
+    found += __popc(mask);
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  stored = found - skip;
+  if (stored < 0) stored = 0;
+  if (stored > MAXSEG) stored = MAXSEG;
+  if (lane == 0) {
+    m->nseg = stored;
+    m->more = (found - skip > MAXSEG) ? 1 : 0;
+  }
+}
+
+// Butterfly reduce-scatter over the 32 lanes of a warp: afterwards lane l holds the
+// reduction of heads [l*N/32, l*N/32 + N/32) in v[0..] (N >= 32), or of head l/2 (N == 16).
+template <int N, bool IS_MAX>
+__device__ __forceinline__ void warp_reduce_scatter(float (&v)[N], int lane) {
+  int n = N;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+    if (n > 1) {
+      const int half = n >> 1;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        if (i < half) {
+          const float send = up ? v[i] : v[i + half];
+          const float keep = up ? v[i + half] : v[i];
+          const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+          v[i] = IS_MAX ? fmaxf(keep, recv) : keep + recv;
+        }
+      }
+      n = half;
+    } else {
+      const float recv = __shfl_xor_sync(0xffffffffu, v[0], o);
+      v[0] = IS_MAX ? fmaxf(v[0], recv) : v[0] + recv;
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void store_scattered(float* dst, const float (&v)[N], int lane) {
+  if constexpr (N >= 32) {
+#pragma unroll
+    for (int i = 0; i < N / 32; ++i) dst[lane * (N / 32) + i] = v[i];
+  } else {
+    if ((lane & 1) == 0) dst[lane >> 1] = v[0];
+  }
+}
+
+// TMEM load of HP consecutive columns of this warp's 32 lanes.
+template <int HP>
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[HP]) {
+#pragma unroll
+  for (int c = 0; c < HP / 16; ++c) tmem_ld16(taddr + 16 * c, v + 16 * c);
+}
+
+template <int HP, int NDC>
+struct Layout {
+  static constexpr int NDB = NDC / 2;                   // 128-dim blocks of O^T
+  static constexpr int Q_BYTES = NDC * HP * 128;        // [NDC][HP][64] bf16
+  static constexpr int RING_BYTES = NST * STAGE_BYTES;
+  static constexpr int P_BYTES = 2 * HP * 128;          // [2][HP][64] bf16 (P^T, K-major)
+  static constexpr int Q_OFF = 0;
+  static constexpr int RING_OFF = Q_OFF + Q_BYTES;
+  static constexpr int P_OFF = RING_OFF + RING_BYTES;
+  static constexpr int MISC_OFF = P_OFF + P_BYTES;
+  static constexpr int SMEM = MISC_OFF + static_cast<int>(sizeof(Misc)) + 1024;  // + alignment
+  static constexpr int TMEM_USED = 2 * HP + NDB * HP;
+  static constexpr uint32_t TMEM_COLS =
+      TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+  static_assert(TMEM_USED <= 512, "tensor memory overflow");
+  static_assert(NDC % 2 == 0 && NST % 2 == 0, "V stage pairs must not straddle the ring end");
+  static_assert(HP % 16 == 0 && HP <= 64, "heads padded to 16, at most 64");
+};
+
+template <int HP, int NDC>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_splitk_kernel(const __grid_constant__ CUtensorMap map_kv,
+                       const __grid_constant__ CUtensorMap map_q, const Args a) {
+  using LY = Layout<HP, NDC>;
+  constexpr int NDB = LY::NDB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + LY::Q_OFF;
+  uint8_t* sRing = smem + LY::RING_OFF;
+  uint8_t* sP = smem + LY::P_OFF;
+  Misc* m = reinterpret_cast<Misc*>(smem + LY::MISC_OFF);
+  volatile int* abort = &m->abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&m->full[i], 1);
+      mbar_init(&m->empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&m->s_full[i], 1);
+      mbar_init(&m->s_free[i], 4);  // one arrive per softmax warp
+    }
+    mbar_init(&m->p_full, 4);
+    mbar_init(&m->pv_done, 1);
+    mbar_init(&m->q_full, 1);
+    mbar_init(&m->q_free, 1);
+    mbar_init(&m->mma_done, 1);
+    m->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&map_kv);
+    prefetch_tensormap(&map_q);
+  }
+  long long U = 0;
+  if (warp == 0) U = warp_total_units(a, lane);
+  if (warp == 1) {
+    tmem_alloc(&m->tmem_base, LY::TMEM_COLS);
+    tmem_relinquish();
+  }
+  // grid-wide split of the batch's units
+  const long long G = gridDim.x;
+  long long us = 0, ue = 0;
+  if (warp == 0) {
+    us = (static_cast<long long>(blockIdx.x) * U) / G;
+    ue = (static_cast<long long>(blockIdx.x + 1) * U) / G;
+    plan_segments(a, us, ue, 0, m, lane);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = m->tmem_base;
+
+  // per-role pipeline counters (persist across segments and batches)
+  int ring_pos = 0;      // stages armed (producer) / consumed (MMA) so far
+  int seg_count = 0;     // segments started by this role
+  int gtile_s = 0;       // S tiles issued / consumed
+  int gtile_o = 0;       // PV tiles issued / P tiles produced
+  const uint64_t evict_first = (warp == 0) ? l2_policy_evict_first() : 0ull;
+
+  for (int batch = 0;; ++batch) {
+    const int nseg = m->nseg;
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        for (int g = 0; g < nseg && !*abort; ++g) {
+          const Seg sg = m->seg[g];
+          const int T = (sg.u1 - sg.u0 + 3) >> 2;
+          if (seg_count > 0 && !mbar_wait(&m->q_free, (seg_count - 1) & 1, abort)) break;
+          mbar_arrive_expect_tx(&m->q_full, NDC * a.H * 128);
+          for (int c = 0; c < NDC; ++c)
+            tma_load_2d(sQ + c * HP * 128, &map_q, &m->q_full, 64 * c, sg.b * a.H);
+          ++seg_count;
+          const int32_t* bt = a.block_table + static_cast<long long>(sg.b) * a.bt_stride;
+          for (int i = 0; i <= T && !*abort; ++i) {
+            for (int kv = 0; kv < 2; ++kv) {
+              // stage order per step i: K of tile i, then V of tile i-1
+              const int tile = kv == 0 ? i : i - 1;
+              if (tile < 0 || tile >= T) continue;
+              const int tu0 = sg.u0 + 4 * tile;
+              const int tu1 = min(tu0 + 4, sg.u1);
+              int ys[4];
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                const int u = (tu0 + r < tu1) ? tu0 + r : tu0;  // pad with a valid unit
+                const int page = __ldg(bt + (u >> 1));
+                int y;
+                if (page < 0 || page >= a.n_pages) {
+                  set_err(a.err, LSA_DEVERR_BAD_PAGE);
+                  y = static_cast<int>(a.n_pages * 128);  // outside the map: zero fill
+                } else {
+                  y = page * 128 + kv * 64 + (u & 1) * UNIT;
+                }
+                ys[r] = y;
+              }
+              for (int c = 0; c < NDC; ++c) {
+                const int st = ring_pos % NST;
+                if (!mbar_wait(&m->empty[st], ((ring_pos / NST) & 1) ^ 1, abort)) break;
+                mbar_arrive_expect_tx(&m->full[st], STAGE_BYTES);
+                uint8_t* dst = sRing + st * STAGE_BYTES;
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                  tma_load_2d_hint(dst + r * (UNIT * 128), &map_kv, &m->full[st], 64 * c, ys[r],
+                                   evict_first);
+                ++ring_pos;
+              }
+            }
+          }
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t IDESC_S = idesc_bf16_f32(128, HP, false, false);
+        constexpr uint32_t IDESC_O = idesc_bf16_f32(128, HP, true, false);
+        const uint32_t q_base = smem_u32(sQ), p_base = smem_u32(sP), ring_base = smem_u32(sRing);
+        for (int g = 0; g < nseg && !*abort; ++g) {
+          const Seg sg = m->seg[g];
+          const int T = (sg.u1 - sg.u0 + 3) >> 2;
+          if (!mbar_wait(&m->q_full, seg_count & 1, abort)) break;
+          tc_fence_after();
+          ++seg_count;
+          bool ok = true;
+          for (int i = 0; i <= T && ok; ++i) {
+            if (i < T) {
+              const int sb = gtile_s & 1;
+              if (gtile_s >= 2 && !mbar_wait(&m->s_free[sb], ((gtile_s >> 1) - 1) & 1, abort)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t d_s = tmem + sb * HP;
+              for (int kb = 0; kb < NDC && ok; ++kb) {
+                const int stg = ring_pos % NST;
+                if (!mbar_wait(&m->full[stg], (ring_pos / NST) & 1, abort)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                const uint32_t st = ring_base + stg * STAGE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  umma_bf16(d_s, sdesc_sw128(st + kk * 32, 16, 1024),
+                            sdesc_sw128(q_base + kb * HP * 128 + kk * 32, 16, 1024), IDESC_S,
+                            (kb | kk) != 0);
+                umma_commit(&m->empty[stg]);
+                ++ring_pos;
+              }
+              if (!ok) break;
+              umma_commit(&m->s_full[sb]);
+              if (i == T - 1) umma_commit(&m->q_free);
+              ++gtile_s;
+            }
+            if (i >= 1) {
+              const int j = i - 1;
+              if (!mbar_wait(&m->p_full, gtile_o & 1, abort)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              for (int db = 0; db < NDB && ok; ++db) {
+                const int st0 = ring_pos % NST;  // even: the pair (st0, st0+1) is adjacent
+                if (!mbar_wait(&m->full[st0], (ring_pos / NST) & 1, abort) ||
+                    !mbar_wait(&m->full[st0 + 1], (ring_pos / NST) & 1, abort)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                const uint32_t st = ring_base + st0 * STAGE_BYTES;
+                const uint32_t d_o = tmem + 2 * HP + db * HP;
+#pragma unroll
+                for (int kk = 0; kk < TILE / 16; ++kk)
+                  umma_bf16(d_o, sdesc_sw128(st + kk * 16 * 128, STAGE_BYTES, 1024),
+                            sdesc_sw128(p_base + (kk >> 2) * HP * 128 + (kk & 3) * 32, 16, 1024),
+                            IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&m->empty[st0]);
+                umma_commit(&m->empty[st0 + 1]);
+                ring_pos += 2;
+              }
+              if (!ok) break;
+              umma_commit(&m->pv_done);
+              ++gtile_o;
+            }
+          }
+        }
+      }
+    } else {
+      // ---------------------------------------------------------------- softmax
+      // Every wait result is folded into the next barrier-with-reduction, so the four
+      // warps always leave together and no named barrier is left half-arrived.
+      const int sw = warp & 3;                 // TMEM sub-partition: rows [32*sw, 32*sw+32)
+      const int t128 = tid - 64;               // 0..127
+      const int row = sw * 32 + lane;          // token row of the tile
+      const uint32_t lane_addr = static_cast<uint32_t>(sw * 32) << 16;
+      bool failed = false;
+      for (int g = 0; g < nseg && !failed; ++g) {
+        const Seg sg = m->seg[g];
+        const int T = (sg.u1 - sg.u0 + 3) >> 2;
+        const int n_ent = __ldg(a.n_entries + sg.b);
+        const int tl = __ldg(a.tail_len + sg.b);
+        float m_run = -INFINITY;               // running max (log2 units) of head t128
+        float lp[HP];
+#pragma unroll
+        for (int h = 0; h < HP; ++h) lp[h] = 0.f;
+        for (int j = 0; j < T; ++j) {
+          const int sb = gtile_s & 1;
+          if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(&m->s_full[sb], (gtile_s >> 1) & 1, abort));
+          tc_fence_after();
+          // validity of this row's token
+          const int u = sg.u0 + 4 * j + sw;
+          bool valid = u < sg.u1;
+          if (valid && (u >> 1) == n_ent - 1) valid = (u & 1) * UNIT + lane < tl;
+          // per-head tile max
+          if (!failed) {
+            float x[HP];
+            tmem_ld_row<HP>(tmem + lane_addr + sb * HP, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < HP; ++h) x[h] = valid ? x[h] : -INFINITY;
+            warp_reduce_scatter<HP, true>(x, lane);
+            store_scattered<HP>(m->red[sw], x, lane);
+          }
+          if (named_bar_any(1, 128, failed)) {
+            failed = true;
+            break;
+          }
+          if (t128 < HP) {
+            const int h = t128;
+            float mt = fmaxf(fmaxf(m->red[0][h], m->red[1][h]), fmaxf(m->red[2][h], m->red[3][h]));
+            mt *= a.scale_log2;
+            float al = 1.f;
+            if (h < a.H && mt > m_run + RESCALE_LOG2) {
+              al = exp2f(m_run - mt);          // 0 when nothing was accumulated yet
+              m_run = mt;
+            }
+            m->m_use[h] = m_run;
+            m->alpha[h] = al;
+          }
+          named_bar_sync(1, 128);
+          float s[HP];
+          tmem_ld_row<HP>(tmem + lane_addr + sb * HP, s);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&m->s_free[sb]);
+          ++gtile_s;
+          bool rescale = false;
+#pragma unroll
+          for (int h = 0; h < HP; ++h) {
+            const float mu = m->m_use[h];
+            const float al = m->alpha[h];
+            rescale |= al < 1.f;
+            const float p = (valid && h < a.H) ? exp2f(fmaf(s[h], a.scale_log2, -mu)) : 0.f;
+            lp[h] = lp[h] * al + p;
+            s[h] = p;
+          }
+          // the previous tile's P . V must be done before P is overwritten or O rescaled
+          if (gtile_o >= 1)
+            failed = !__all_sync(0xffffffffu, mbar_wait(&m->pv_done, (gtile_o - 1) & 1, abort));
+          if (failed) continue;                // the next barrier reports it to all warps
+          tc_fence_after();
+          if (rescale && j > 0) {
+#pragma unroll
+            for (int db = 0; db < NDB; ++db) {
+#pragma unroll
+              for (int c = 0; c < HP / 16; ++c) {
+                const uint32_t ta = tmem + lane_addr + 2 * HP + db * HP + 16 * c;
+                float o[16];
+                tmem_ld16(ta, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] *= m->alpha[16 * c + i];
+                tmem_st16(ta, o);
+              }
+            }
+            tmem_wait_st();
+          }
+          // P^T (K-major: row = head, 128 tokens in two 64-token chunks), bf16
+          {
+            uint8_t* pc = sP + (row >> 6) * HP * 128;
+            const uint32_t byte_in_row = (row & 63) * 2;
+#pragma unroll
+            for (int h = 0; h < HP; ++h) {
+              const __nv_bfloat16 v = __float2bfloat16_rn(s[h]);
+              *reinterpret_cast<__nv_bfloat16*>(pc + sw128_offset(h, byte_in_row)) = v;
+            }
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&m->p_full);
+          ++gtile_o;
+        }
+        if (named_bar_any(1, 128, failed)) {
+          failed = true;
+          break;
+        }
+        // ------------------------------------------------------- segment epilogue
+        failed = !__all_sync(0xffffffffu, mbar_wait(&m->pv_done, (gtile_o - 1) & 1, abort));
+        tc_fence_after();
+        if (!failed) {
+          warp_reduce_scatter<HP, false>(lp, lane);
+          store_scattered<HP>(m->red[sw], lp, lane);
+        }
+        if (named_bar_any(1, 128, failed)) {
+          failed = true;
+          break;
+        }
+        const long long slot = static_cast<long long>(blockIdx.x) + sg.b;
+        if (t128 < a.H) {
+          const int h = t128;
+          const float l = m->red[0][h] + m->red[1][h] + m->red[2][h] + m->red[3][h];
+          a.part_ml[(slot * a.H + h) * 2 + 0] = m_run;
+          a.part_ml[(slot * a.H + h) * 2 + 1] = l;
+        }
+        float* po = a.part_o + slot * a.H * a.d;
+#pragma unroll
+        for (int db = 0; db < NDB; ++db) {
+#pragma unroll
+          for (int c = 0; c < HP / 16; ++c) {
+            float o[16];
+            tmem_ld16(tmem + lane_addr + 2 * HP + db * HP + 16 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int h = 16 * c + i;
+              if (h < a.H) po[static_cast<long long>(h) * a.d + db * 128 + row] = o[i];
+            }
+          }
+        }
+        tc_fence_before();
+        named_bar_sync(1, 128);
+      }
+    }
+
+    // ------------------------------------------------------------ next batch
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (!m->more || *abort) break;
+    __syncthreads();
+    if (warp == 0) plan_segments(a, us, ue, (batch + 1) * MAXSEG, m, lane);
+    __syncthreads();
+  }
+
+  // ---------------------------------------------------------------- teardown
+  if (*abort) {
+    if (tid == 0) set_err(a.err, LSA_DEVERR_TIMEOUT);
+    // the producer waits (bounded) for its own copies still in flight
+    if (warp == 0 && lane == 0) {
+      for (int k = max(0, ring_pos - NST); k < ring_pos; ++k)
+        mbar_wait(&m->full[k % NST], (k / NST) & 1, nullptr);
+      if (seg_count > 0) mbar_wait(&m->q_full, (seg_count - 1) & 1, nullptr);
+    }
+    // the MMA thread waits (bounded) for its own tensor-core work
+    if (warp == 1 && lane == 0) {
+      umma_commit(&m->mma_done);
+      mbar_wait(&m->mma_done, 0, nullptr);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, LY::TMEM_COLS);
+}
+
+// Log-sum-exp merge of the partial results of every segment of sequence b, head h:
+//   M = max_k m_k,  out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k   (m in log2 units)
+// The segments of b are the CTAs whose unit ranges meet b's units; slot = CTA + b.
+// grid (H, B), d/4 threads, each owning 4 consecutive dimensions.
+__global__ void __launch_bounds__(128) attn_merge_kernel(const Args a, int G, uint16_t* out) {
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  __shared__ long long s_tot[2];
+  __shared__ long long s_part[4][2];
+  // prefix of units before b, and the batch total
+  long long before = 0, total = 0;
+  for (int i = tid; i < a.B; i += blockDim.x) {
+    const int u = seq_units(a, i);
+    total += u;
+    if (i < b) before += u;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+  }
+  if ((tid & 31) == 0) {
+    s_part[tid >> 5][0] = total;
+    s_part[tid >> 5][1] = before;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    long long t = 0, bf = 0;
+    for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) {
+      t += s_part[w][0];
+      bf += s_part[w][1];
+    }
+    s_tot[0] = t;
+    s_tot[1] = bf;
+    if (h == 0 && seq_malformed(a, b)) set_err(a.err, LSA_DEVERR_BAD_SIZE);
+  }
+  __syncthreads();
+  const long long U = s_tot[0], P = s_tot[1];
+  const int ub = seq_units(a, b);
+  const int d0 = tid * 4;
+  uint16_t* dst = out + (static_cast<long long>(b) * a.H + h) * a.d + d0;
+  if (d0 >= a.d) return;
+  if (ub == 0) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+    return;
+  }
+  // CTA holding unit u: the largest c with floor(c*U/G) <= u
+  const long long c_lo = ((P + 1) * G - 1) / U;
+  const long long c_hi = ((P + ub) * G - 1) / U;
+  // CTAs with an empty unit range (when the grid outnumbers the units) hold no slot
+  auto empty_cta = [&](long long c) { return (c * U) / G == ((c + 1) * U) / G; };
+  float M = -INFINITY;
+  for (long long c = c_lo; c <= c_hi; ++c)
+    if (!empty_cta(c)) M = fmaxf(M, a.part_ml[((c + b) * a.H + h) * 2]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.f;
+  for (long long c = c_lo; c <= c_hi; ++c) {
+    if (empty_cta(c)) continue;
+    const long long slot = c + b;
+    const float w = exp2f(a.part_ml[(slot * a.H + h) * 2] - M);
+    lsum += w * a.part_ml[(slot * a.H + h) * 2 + 1];
+    const float4 o = *reinterpret_cast<const float4*>(a.part_o + (slot * a.H + h) * a.d + d0);
+    acc.x += w * o.x;
+    acc.y += w * o.y;
+    acc.z += w * o.z;
+    acc.w += w * o.w;
+  }
+  const float inv = 1.f / lsum;
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2 pk;
+  pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(dst) = pk;
+}
+
+}  // namespace attn
+}  // namespace lsa
+
+// ------------------------------------------------------------------------ host side
+namespace {
+
+using lsa::attn::Args;
+
+size_t attn_ws_bytes(int B, int H, int d, int n_sm) {
+  const size_t slots = static_cast<size_t>(n_sm) + static_cast<size_t>(B);
+  return slots * static_cast<size_t>(H) * (static_cast<size_t>(d) + 2) * sizeof(float);
+}
+
+template <int HP, int NDC>
+lsa_status launch_attn(const CUtensorMap& mkv, const CUtensorMap& mq, const Args& a, int G,
+                       cudaStream_t stream) {
+  using LY = lsa::attn::Layout<HP, NDC>;
+  auto kern = lsa::attn::attn_splitk_kernel<HP, NDC>;
+  static int configured_device = -1;  // the attribute is per device and function
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LSA_ERR_CUDA;
+  if (configured_device != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM) !=
+        cudaSuccess)
+      return LSA_ERR_CUDA;
+    configured_device = dev;
+  }
+  kern<<<G, lsa::attn::NTHREADS, LY::SMEM, stream>>>(mkv, mq, a);
+  return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}
+
+template <int HP>
+lsa_status dispatch_d(const CUtensorMap& mkv, const CUtensorMap& mq, const Args& a, int G,
+                      cudaStream_t s) {
+  switch (a.d) {
+    case 128: return launch_attn<HP, 2>(mkv, mq, a, G, s);
+    case 256: return launch_attn<HP, 4>(mkv, mq, a, G, s);
+    case 384: return launch_attn<HP, 6>(mkv, mq, a, G, s);
+    case 512: return launch_attn<HP, 8>(mkv, mq, a, G, s);
+    default: return LSA_ERR_INVALID_ARG;
+  }
+}
+
+}  // namespace
+
+extern "C" size_t lsa_decode_attn_workspace_size(int32_t B, int32_t H, int32_t d, int32_t n_sm) {
+  if (B <= 0 || H <= 0 || d <= 0 || n_sm <= 0) return 0;
+  return attn_ws_bytes(B, H, d, n_sm);
+}
+
+extern "C" lsa_status lsa_decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pages,
+                                      const int32_t* block_table, int32_t bt_stride,
+                                      const int32_t* n_entries, const int32_t* tail_len,
+                                      int32_t B, int32_t H, int32_t d, float scale, uint16_t* out,
+                                      void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+  if (!q || !hbm_pool || !block_table || !n_entries || !tail_len || !out || !ws || !err)
+    return LSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || H > 64 || bt_stride <= 0 || n_pages <= 0) return LSA_ERR_INVALID_ARG;
+  if (d != 128 && d != 256 && d != 384 && d != 512) return LSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return LSA_ERR_INVALID_ARG;
+  if (n_pages > (int64_t(1) << 23)) return LSA_ERR_INVALID_ARG;  // page rows must fit in int32
+  if (static_cast<int64_t>(B) * H > (int64_t(1) << 30)) return LSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(hbm_pool) |
+       reinterpret_cast<uintptr_t>(ws)) & 15u)
+    return LSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(out) & 7u) != 0) return LSA_ERR_INVALID_ARG;
+  const int G = lsa_host::sm_count();
+  if (G <= 0) return LSA_ERR_CUDA;
+  if (ws_bytes < attn_ws_bytes(B, H, d, G)) return LSA_ERR_INVALID_ARG;
+  const int HP = (H + 15) / 16 * 16;
+  const int HPk = HP <= 16 ? 16 : HP <= 32 ? 32 : 64;
+
+  CUtensorMap mkv, mq;
+  lsa_status st = lsa_host::encode_tiled_2d(&mkv, hbm_pool, d, static_cast<uint64_t>(n_pages) * 128,
+                                            static_cast<uint64_t>(d) * 2, 64, lsa::attn::UNIT,
+                                            CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != LSA_OK) return st;
+  st = lsa_host::encode_tiled_2d(&mq, q, d, static_cast<uint64_t>(B) * H,
+                                 static_cast<uint64_t>(d) * 2, 64, H,
+                                 CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != LSA_OK) return st;
+
+  Args a;
+  a.block_table = block_table;
+  a.n_entries = n_entries;
+  a.tail_len = tail_len;
+  a.part_o = static_cast<float*>(ws);
+  a.part_ml = a.part_o + (static_cast<size_t>(G) + B) * H * d;
+  a.err = err;
+  a.n_pages = n_pages;
+  a.bt_stride = bt_stride;
+  a.B = B;
+  a.H = H;
+  a.d = d;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (HPk) {
+    case 16: st = dispatch_d<16>(mkv, mq, a, G, s); break;
+    case 32: st = dispatch_d<32>(mkv, mq, a, G, s); break;
+    default: st = dispatch_d<64>(mkv, mq, a, G, s); break;
+  }
+  if (st != LSA_OK) return st;
+  lsa::attn::attn_merge_kernel<<<dim3(H, B), d / 4, 0, s>>>(a, G, out);
+  return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}

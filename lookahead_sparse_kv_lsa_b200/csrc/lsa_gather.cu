@@ -1,0 +1,339 @@
+// Cold pool -> HBM pool gather of the kept blocks, block-table construction, and the
+// small per-pass / per-step kernels of the decode loop driver.
+//
+// Section 2, step 3 of "FlashMemory-DeepSeek-V4 Explained" (zhichai.net): the blocks
+// the indexer keeps are moved from the CPU cold pool to the GPU before the next 64
+// decode steps attend to them. The pool pages are read by the SMs straight from pinned
+// host memory (mapped into the device address space) with 16-byte loads, eight in
+// flight per thread, so the selected ids never travel back to the host.
+#include "lsa_common.cuh"
+
+namespace lsa {
+namespace gth {
+
+constexpr int THREADS = 256;
+constexpr int MAX_B = 4096;          // sequences per call (prefix sums live in shared memory)
+constexpr int UNROLL = 8;
+
+struct GatherArgs {
+  const uint16_t* host_pool;
+  long long host_blocks;
+  const int64_t* host_blk_off;
+  const int32_t* sel_ids;
+  const int32_t* sel_cnt;
+  const int32_t* res_pages;
+  const int32_t* n_res;
+  uint16_t* hbm_pool;
+  long long n_pages;
+  int32_t* block_table;
+  int32_t* n_entries;
+  int32_t* err;
+  int cap, res_stride, B, d, sel_page_base, sel_page_count, bt_stride;
+};
+
+// Copy one [2][64][d] bf16 block (256*d bytes) with the whole CTA.
+__device__ __forceinline__ void copy_block(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                           int n16) {
+  for (int i0 = threadIdx.x; i0 < n16; i0 += THREADS * UNROLL) {
+    uint4 v[UNROLL];
+#pragma unroll
+    for (int k = 0; k < UNROLL; ++k) {
+      const int i = i0 + k * THREADS;
+      if (i < n16) v[k] = __ldcs(src + i);
+    }
+#pragma unroll
+    for (int k = 0; k < UNROLL; ++k) {
+      const int i = i0 + k * THREADS;
+      if (i < n16) __stcs(dst + i, v[k]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(THREADS) gather_kernel(const GatherArgs a) {
+  __shared__ int s_pref[MAX_B + 1];  // exclusive prefix of the kept-block counts
+  __shared__ int s_warp[THREADS / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int carry = 0;
+  for (int b0 = 0; b0 < a.B; b0 += THREADS) {
+    const int b = b0 + tid;
+    int c = 0;
+    if (b < a.B) {
+      c = __ldg(a.sel_cnt + b);
+      c = c < 0 ? 0 : (c > a.cap ? a.cap : c);
+    }
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int before = carry;
+    for (int k = 0; k < warp; ++k) before += s_warp[k];
+    if (b < a.B) s_pref[b] = before + incl - c;
+    int tot = 0;
+    for (int k = 0; k < THREADS / 32; ++k) tot += s_warp[k];
+    carry += tot;
+    __syncthreads();
+  }
+  if (tid == 0) s_pref[a.B] = carry;
+  __syncthreads();
+  const int total = s_pref[a.B];
+
+  // resident pages (window, tail last) after each sequence's kept blocks
+  for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
+    const int cnt = s_pref[b + 1] - s_pref[b];
+    int nr = __ldg(a.n_res + b);
+    if (nr < 0 || nr > a.res_stride || cnt + nr > a.bt_stride) {
+      if (tid == 0) set_err(a.err, LSA_DEVERR_BAD_SIZE);
+      nr = 0;
+    }
+    int32_t* bt = a.block_table + static_cast<long long>(b) * a.bt_stride;
+    for (int i = tid; i < nr; i += THREADS)
+      bt[cnt + i] = __ldg(a.res_pages + static_cast<long long>(b) * a.res_stride + i);
+    if (tid == 0) a.n_entries[b] = cnt + nr;
+  }
+
+  // kept blocks: item k goes to page sel_page_base + k
+  const int n16 = 16 * a.d;
+  for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    int lo = 0, hi = a.B - 1;  // last b with s_pref[b] <= item
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pref[mid] <= item) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo, j = item - s_pref[b];
+    const int c = __ldg(a.sel_ids + static_cast<long long>(b) * a.cap + j);
+    const long long page = static_cast<long long>(a.sel_page_base) + item;
+    const long long src = __ldg(a.host_blk_off + b) + c;
+    const bool fits = item < a.sel_page_count && page < a.n_pages;
+    const bool valid = c >= 0 && src >= 0 && src < a.host_blocks;
+    if (tid == 0) {
+      if (!fits) set_err(a.err, LSA_DEVERR_POOL_CAPACITY);
+      if (!valid) set_err(a.err, LSA_DEVERR_BAD_PAGE);
+      a.block_table[static_cast<long long>(b) * a.bt_stride + j] =
+          (fits && valid) ? static_cast<int32_t>(page) : -1;
+    }
+    if (!fits || !valid) continue;
+    copy_block(reinterpret_cast<const uint4*>(a.host_pool + src * 128 * a.d),
+               reinterpret_cast<uint4*>(a.hbm_pool + page * 128 * a.d), n16);
+  }
+}
+
+// ----------------------------------------------------------- decode loop driver kernels
+struct StepArgs {
+  const int32_t* nb0;
+  const int64_t* host_blk_off;   // [B+1]
+  uint16_t* host_pool;
+  long long host_blocks;
+  uint16_t* hbm_pool;
+  int32_t* n_cand;
+  int32_t* res_pages;
+  int32_t* n_res;
+  int32_t* tail_len;
+  int32_t* err;
+  int B, d, wb, max_cand;
+};
+
+// window ring page of block j of sequence b
+__device__ __forceinline__ long long ring_page(const StepArgs& a, int b, long long j) {
+  return static_cast<long long>(b) * (a.wb + 1) + j % (a.wb + 1);
+}
+
+// Pass p set-up (one CTA per sequence): candidate count, resident page list (window
+// blocks oldest first, then the new tail page), and a zeroed tail page.
+__global__ void __launch_bounds__(THREADS) pass_setup_kernel(const StepArgs a, int p) {
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const long long nb = static_cast<long long>(__ldg(a.nb0 + b)) + p;
+  const long long first = nb - a.wb > 0 ? nb - a.wb : 0;
+  if (tid == 0) {
+    long long nc = nb - a.wb;
+    if (nc < 0) nc = 0;
+    if (nc > a.max_cand) {
+      set_err(a.err, LSA_DEVERR_BAD_SIZE);
+      nc = a.max_cand;
+    }
+    a.n_cand[b] = static_cast<int32_t>(nc);
+    a.n_res[b] = static_cast<int32_t>(nb - first + 1);
+    a.tail_len[b] = 0;
+  }
+  for (long long i = tid; i < nb - first + 1; i += THREADS)
+    a.res_pages[static_cast<long long>(b) * (a.wb + 1) + i] =
+        static_cast<int32_t>(ring_page(a, b, first + i));
+  uint4* tail = reinterpret_cast<uint4*>(a.hbm_pool + ring_page(a, b, nb) * 128 * a.d);
+  for (int i = tid; i < 16 * a.d; i += THREADS) tail[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Step s of pass p: write the new token's K and V into slot s of the tail page, write it
+// through to the cold pool, and set tail_len = s + 1. One CTA per sequence, d/8 threads.
+__global__ void append_kernel(const StepArgs a, int p, int s, const uint16_t* __restrict__ k_new,
+                              const uint16_t* __restrict__ v_new) {
+  const int b = blockIdx.x, t = threadIdx.x;
+  const long long nb = static_cast<long long>(__ldg(a.nb0 + b)) + p;
+  const long long page = ring_page(a, b, nb);
+  const uint4 k = reinterpret_cast<const uint4*>(k_new + static_cast<long long>(b) * a.d)[t];
+  const uint4 v = reinterpret_cast<const uint4*>(v_new + static_cast<long long>(b) * a.d)[t];
+  reinterpret_cast<uint4*>(a.hbm_pool + (page * 128 + s) * a.d)[t] = k;
+  reinterpret_cast<uint4*>(a.hbm_pool + (page * 128 + 64 + s) * a.d)[t] = v;
+  const long long hb = __ldg(a.host_blk_off + b) + nb;
+  if (hb < __ldg(a.host_blk_off + b + 1) && hb < a.host_blocks) {
+    reinterpret_cast<uint4*>(a.host_pool + (hb * 128 + s) * a.d)[t] = k;
+    reinterpret_cast<uint4*>(a.host_pool + (hb * 128 + 64 + s) * a.d)[t] = v;
+  } else if (t == 0) {
+    set_err(a.err, LSA_DEVERR_BAD_PAGE);
+  }
+  if (t == 0) a.tail_len[b] = s + 1;
+}
+
+// Load the window blocks of pass p from the cold pool into the rings. grid (wb, B).
+__global__ void __launch_bounds__(THREADS) load_window_kernel(const StepArgs a, int p) {
+  const int i = blockIdx.x, b = blockIdx.y;
+  const long long nb = static_cast<long long>(__ldg(a.nb0 + b)) + p;
+  const long long blk = nb - a.wb + i;
+  if (blk < 0) return;
+  const long long src = __ldg(a.host_blk_off + b) + blk;
+  if (src >= __ldg(a.host_blk_off + b + 1) || src >= a.host_blocks) {
+    if (threadIdx.x == 0) set_err(a.err, LSA_DEVERR_BAD_PAGE);
+    return;
+  }
+  copy_block(reinterpret_cast<const uint4*>(a.host_pool + src * 128 * a.d),
+             reinterpret_cast<uint4*>(a.hbm_pool + ring_page(a, b, blk) * 128 * a.d), 16 * a.d);
+}
+
+}  // namespace gth
+}  // namespace lsa
+
+// ------------------------------------------------------------------------ host side
+namespace lsa_host {
+
+// Device-visible address of pinned host memory (the same pointer under unified
+// addressing); nullptr if `p` is not page-locked host memory.
+const void* mapped_host_ptr(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (at.type != cudaMemoryTypeHost || at.devicePointer == nullptr) return nullptr;
+  return at.devicePointer;
+}
+
+}  // namespace lsa_host
+
+extern "C" lsa_status lsa_gather(const uint16_t* host_pool, int64_t host_blocks,
+                                 const int64_t* host_blk_off, const int32_t* sel_ids,
+                                 const int32_t* sel_cnt, int32_t cap, const int32_t* res_pages,
+                                 const int32_t* n_res, int32_t res_stride, int32_t B, int32_t d,
+                                 uint16_t* hbm_pool, int64_t n_pages, int32_t sel_page_base,
+                                 int32_t sel_page_count, int32_t* block_table, int32_t bt_stride,
+                                 int32_t* n_entries, int32_t* err, void* stream) {
+  if (!host_pool || !host_blk_off || !sel_cnt || !res_pages || !n_res || !hbm_pool ||
+      !block_table || !n_entries || !err)
+    return LSA_ERR_INVALID_ARG;
+  if (cap > 0 && !sel_ids) return LSA_ERR_INVALID_ARG;
+  if (B <= 0 || B > lsa::gth::MAX_B || d <= 0 || d % 8 != 0 || cap < 0 || res_stride < 0 ||
+      host_blocks <= 0 || n_pages <= 0 || sel_page_base < 0 || sel_page_count < 0 ||
+      bt_stride < cap + res_stride)
+    return LSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(sel_page_base) + sel_page_count > n_pages) return LSA_ERR_INVALID_ARG;
+  const void* hp = lsa_host::mapped_host_ptr(host_pool);
+  if (hp == nullptr) return LSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(hp) | reinterpret_cast<uintptr_t>(hbm_pool)) & 15u)
+    return LSA_ERR_INVALID_ARG;
+  lsa::gth::GatherArgs a;
+  a.host_pool = static_cast<const uint16_t*>(hp);
+  a.host_blocks = host_blocks;
+  a.host_blk_off = host_blk_off;
+  a.sel_ids = sel_ids;
+  a.sel_cnt = sel_cnt;
+  a.res_pages = res_pages;
+  a.n_res = n_res;
+  a.hbm_pool = hbm_pool;
+  a.n_pages = n_pages;
+  a.block_table = block_table;
+  a.n_entries = n_entries;
+  a.err = err;
+  a.cap = cap;
+  a.res_stride = res_stride;
+  a.B = B;
+  a.d = d;
+  a.sel_page_base = sel_page_base;
+  a.sel_page_count = sel_page_count;
+  a.bt_stride = bt_stride;
+  const int G = lsa_host::sm_count();
+  if (G <= 0) return LSA_ERR_CUDA;
+  lsa::gth::gather_kernel<<<2 * G, lsa::gth::THREADS, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ decode loop driver
+namespace {
+lsa::gth::StepArgs step_args(const lsa_state* st, const void* host_dev) {
+  lsa::gth::StepArgs a;
+  a.nb0 = st->nb0;
+  a.host_blk_off = st->host_blk_off;
+  a.host_pool = static_cast<uint16_t*>(const_cast<void*>(host_dev));
+  a.host_blocks = st->host_blocks;
+  a.hbm_pool = st->hbm_pool;
+  a.n_cand = st->n_cand;
+  a.res_pages = st->res_pages;
+  a.n_res = st->n_res;
+  a.tail_len = st->tail_len;
+  a.err = st->err;
+  a.B = st->B;
+  a.d = st->d;
+  a.wb = st->W / LSA_BLOCK;
+  a.max_cand = st->max_cand;
+  return a;
+}
+}  // namespace
+
+extern "C" lsa_status lsa_load_window(const lsa_state* st, int32_t pass, void* stream) {
+  const lsa_status v = lsa_state_check(st);
+  if (v != LSA_OK) return v;
+  if (pass < 0) return LSA_ERR_INVALID_ARG;
+  const void* hp = lsa_host::mapped_host_ptr(st->host_pool);
+  if (hp == nullptr) return LSA_ERR_INVALID_ARG;
+  const lsa::gth::StepArgs a = step_args(st, hp);
+  if (a.wb == 0) return LSA_OK;
+  lsa::gth::load_window_kernel<<<dim3(a.wb, st->B), lsa::gth::THREADS, 0,
+                                 static_cast<cudaStream_t>(stream)>>>(a, pass);
+  return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}
+
+extern "C" lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t* h,
+                               const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                               uint16_t* out, void* stream) {
+  lsa_status v = lsa_state_check(st);
+  if (v != LSA_OK) return v;
+  if (step < 0 || step / LSA_TAU > (int64_t(1) << 30) || !q || !k_new || !v_new || !out)
+    return LSA_ERR_INVALID_ARG;
+  const int p = static_cast<int>(step / LSA_TAU), s = static_cast<int>(step % LSA_TAU);
+  if (s == 0 && !h) return LSA_ERR_INVALID_ARG;
+  const void* hp = lsa_host::mapped_host_ptr(st->host_pool);
+  if (hp == nullptr) return LSA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const lsa::gth::StepArgs a = step_args(st, hp);
+  const int wb1 = a.wb + 1;
+  if (s == 0) {
+    lsa::gth::pass_setup_kernel<<<st->B, lsa::gth::THREADS, 0, cs>>>(a, p);
+    if (cudaGetLastError() != cudaSuccess) return LSA_ERR_CUDA;
+    v = lsa_index(h, st->w_q, st->bias, st->k_idx, st->kidx_off, st->n_cand, st->B, st->L, st->D,
+                  st->d_i, st->max_cand, st->sel_ids, st->sel_cnt, st->cap, nullptr, nullptr,
+                  st->index_ws, st->index_ws_bytes, st->err, stream);
+    if (v != LSA_OK) return v;
+    const int64_t base = static_cast<int64_t>(st->B) * wb1;
+    v = lsa_gather(st->host_pool, st->host_blocks, st->host_blk_off, st->sel_ids, st->sel_cnt,
+                   st->cap, st->res_pages, st->n_res, wb1, st->B, st->d, st->hbm_pool,
+                   st->n_pages, static_cast<int32_t>(base),
+                   static_cast<int32_t>(st->n_pages - base), st->block_table, st->bt_stride,
+                   st->n_entries, st->err, stream);
+    if (v != LSA_OK) return v;
+  }
+  lsa::gth::append_kernel<<<st->B, st->d / 8, 0, cs>>>(a, p, s, k_new, v_new);
+  if (cudaGetLastError() != cudaSuccess) return LSA_ERR_CUDA;
+  return lsa_decode_attn(q, st->hbm_pool, st->n_pages, st->block_table, st->bt_stride,
+                         st->n_entries, st->tail_len, st->B, st->H, st->d, st->scale, out,
+                         st->attn_ws, st->attn_ws_bytes, st->err, stream);
+}

@@ -48,7 +48,8 @@ def _randn_bf16(shape, gen: torch.Generator, std: float = 1.0) -> torch.Tensor:
 class Workload:
     """All inputs of one LSA decode run (one config)."""
 
-    def __init__(self, cfg: LsaConfig, pin: bool = False, threads: Optional[int] = None):
+    def __init__(self, cfg: LsaConfig, pin: bool = False, threads: Optional[int] = None,
+                 with_pool: bool = True):
         self.cfg = cfg
         B, blk = cfg.B, cfg.block
         # context lengths (tokens at pass 0) and per-sequence bias
@@ -80,9 +81,11 @@ class Workload:
         for b in range(B):
             self.k_idx[off[b]:off[b + 1]] = _randn_bf16(
                 (int(self.nb_final[b]), cfg.d_i), _gen(cfg.seed, "k_idx", b))
-        self.host_pool = torch.empty((self.total_blocks, 2, blk, cfg.d), dtype=torch.bfloat16,
-                                     pin_memory=pin)
-        self._fill_pool(threads)
+        self.host_pool = None
+        if with_pool:
+            self.host_pool = torch.empty((self.total_blocks, 2, blk, cfg.d), dtype=torch.bfloat16,
+                                         pin_memory=pin)
+            self._fill_pool(threads)
 
     # -- cold pool ---------------------------------------------------------------
     def _fill_pool(self, threads):

@@ -1,0 +1,103 @@
+"""GPU parity of lsa_index (projection, scoring, sign test, OR, compaction) against the
+oracle, at the full sizes of every workload (the indexer is cheap for the oracle)."""
+import numpy as np
+import pytest
+import torch
+
+import lookahead_sparse_kv_lsa_b200 as lsa
+import lsa_inputs as LI
+import oracle
+from gpu_util import LOGIT_ABS, NEAR_TIE, bits, compare_selection
+
+pytestmark = pytest.mark.gpu
+
+CONFIGS = {
+    "tiny_16k": LI.tiny,
+    "mid_b8_128k": LI.mid_batch,
+    "long_b4_512k": LI.long_ctx,
+    "1m_b15": lambda: LI.one_million(-1.5),
+    "1m_b20": lambda: LI.one_million(-2.0),
+    "1m_b25": lambda: LI.one_million(-2.5),
+    "ragged_b64": LI.ragged_mix,
+}
+
+
+def run_index(wl, p, cap=None, n_cand=None):
+    dev = torch.device("cuda")
+    c = wl.cfg
+    B, L = c.B, c.L
+    if n_cand is None:
+        n_cand = [oracle.n_candidates(int(x), c.W) for x in wl.ctx_at(p)]
+    max_cand = max(1, max(n_cand))
+    cap = max_cand if cap is None else cap
+    h = wl.h(p).to(dev)
+    sel_ids = torch.full((B, max(1, cap)), -1, dtype=torch.int32, device=dev)
+    sel_cnt = torch.full((B,), -1, dtype=torch.int32, device=dev)
+    logits = torch.full((L, B, max_cand), float("nan"), device=dev)
+    mask = torch.zeros((L + 1, B, (max_cand + 31) // 32), dtype=torch.int32, device=dev)
+    ws = torch.zeros(lsa.index_workspace_size(B, L, c.d_i, max_cand), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    lsa.lsa_index(h, wl.w_q.to(dev), torch.from_numpy(wl.bias).to(dev), wl.k_idx.to(dev),
+                  torch.from_numpy(wl.blk_off[:B]).to(dev),
+                  torch.tensor(n_cand, dtype=torch.int32, device=dev), max_cand, sel_ids, sel_cnt,
+                  ws, err, logits=logits, layer_mask=mask)
+    torch.cuda.synchronize()
+    return (sel_ids.cpu(), sel_cnt.cpu(), logits.cpu().numpy(), mask.cpu().numpy().view(np.uint32),
+            int(err.item()), n_cand)
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_index_matches_oracle(cuda_ok, name):
+    wl = LI.Workload(CONFIGS[name](), with_pool=False)
+    c = wl.cfg
+    for p in range(c.passes):
+        ids, cnt, z_gpu, mask, err, n_cand = run_index(wl, p)
+        assert err == 0
+        hb = bits(wl.h(p))
+        n_near = 0
+        for b in range(c.B):
+            nc = n_cand[b]
+            ref_ids, z_ref = oracle.index_pass(bits(wl.w_q), hb[:, b], bits(wl.seq_k_idx(b)[:nc]),
+                                               float(wl.bias[b]))
+            dz = np.abs(z_gpu[:, b, :nc] - z_ref)
+            assert dz.max(initial=0.0) <= LOGIT_ABS, (name, b, dz.max())
+            got = ids[b, :int(cnt[b])].tolist()
+            n_near += len(compare_selection(got, ref_ids, z_ref, "%s p%d b%d" % (name, p, b)))
+            # per-layer bits and the OR word agree with the kernel's own logits exactly
+            for l in range(c.L + 1):
+                bitv = np.unpackbits(mask[l, b].view(np.uint8), bitorder="little")[:nc].astype(bool)
+                zz = z_gpu[:, b, :nc]
+                expect = (zz > 0).any(axis=0) if l == c.L else zz[l] > 0
+                assert np.array_equal(bitv, expect)
+            assert got == np.flatnonzero((z_gpu[:, b, :nc] > 0).any(axis=0)).tolist()
+        # near ties are rare: ~2e-3 * phi(bias) * 3 per candidate
+        assert n_near <= max(3, 0.01 * sum(n_cand))
+
+
+def test_capacity_overflow_flagged(cuda_ok):
+    wl = LI.Workload(LI.tiny(), with_pool=False)
+    ids_full, cnt_full, *_ = run_index(wl, 0)
+    n = int(cnt_full[0])
+    assert n > 4
+    ids, cnt, _, _, err, _ = run_index(wl, 0, cap=4)
+    assert err & lsa._lib.DEVERR_SEL_CAPACITY
+    assert int(cnt[0]) == 4 and ids[0, :4].tolist() == ids_full[0, :4].tolist()
+
+
+def test_no_candidates(cuda_ok):
+    wl = LI.Workload(LI.tiny(), with_pool=False)
+    ids, cnt, _, _, err, _ = run_index(wl, 0, n_cand=[0])
+    assert err == 0 and int(cnt[0]) == 0
+
+
+def test_all_and_none_kept(cuda_ok):
+    cfg = LI.tiny()
+    for bias, expect_all in ((1e4, True), (-1e4, False)):
+        cfg.bias = [bias]
+        wl = LI.Workload(cfg, with_pool=False)
+        ids, cnt, _, _, err, n_cand = run_index(wl, 0)
+        assert err == 0
+        if expect_all:
+            assert ids[0, :int(cnt[0])].tolist() == list(range(n_cand[0]))
+        else:
+            assert int(cnt[0]) == 0

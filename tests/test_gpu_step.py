@@ -1,0 +1,108 @@
+"""GPU parity of the whole decode loop (lsa_step: index + gather every 64 steps, append +
+attention every step) against the oracle's loop, on every workload: in full at the tiny
+size and scaled-down sizes, and on sampled steps and heads at the full 1M-token size."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import lookahead_sparse_kv_lsa_b200 as lsa
+import lsa_inputs as LI
+import oracle
+from gpu_util import bits, compare_attention, compare_selection
+
+pytestmark = pytest.mark.gpu
+
+
+def build_decoder(wl):
+    dev = torch.device("cuda")
+    c = wl.cfg
+    max_cand = max(1, max(oracle.n_candidates(int(x), c.W) for x in wl.ctx_at(c.passes - 1)))
+    return lsa.LsaDecoder(wl.w_q.to(dev), wl.k_idx.to(dev), wl.blk_off[:c.B],
+                          torch.from_numpy(wl.bias).to(dev), wl.host_pool, wl.blk_off, wl.nb0,
+                          W=c.W, H=c.H, cap=max_cand, max_cand=max_cand, scale=c.scale)
+
+
+def run_loop(wl, keep_steps):
+    """Runs every step of every pass; returns {(p, s): out}, [per-pass (ids, cnt)]."""
+    dev = torch.device("cuda")
+    c = wl.cfg
+    dec = build_decoder(wl)
+    dec.load_window(0)
+    outs, sels = {}, []
+    out = torch.empty((c.B, c.H, c.d), dtype=torch.bfloat16, device=dev)
+    for p in range(c.passes):
+        h = wl.h(p).to(dev)
+        for s in range(c.tau):
+            k, v = wl.kv_new(p, s)
+            dec.step(p * c.tau + s, h if s == 0 else None, wl.q(p, s).to(dev), k.to(dev),
+                     v.to(dev), out)
+            if s == 0:
+                sels.append((dec.sel_ids.cpu().clone(), dec.sel_cnt.cpu().clone()))
+            if s in keep_steps:
+                outs[(p, s)] = out.cpu().clone()
+    torch.cuda.synchronize()
+    assert dec.read_err() == 0, "device error word %d" % dec.read_err()
+    return outs, sels
+
+
+def check_loop(wl, keep_steps, heads=None):
+    c = wl.cfg
+    outs, sels = run_loop(wl, keep_steps)
+    wq = bits(wl.w_q)
+    for p in range(c.passes):
+        hb = bits(wl.h(p))
+        ids_gpu, cnt_gpu = sels[p]
+        for b in range(c.B):
+            n_ctx = int(wl.ctx_at(p)[b])
+            nc = oracle.n_candidates(n_ctx, c.W)
+            ref_ids, z = oracle.index_pass(wq, hb[:, b], bits(wl.seq_k_idx(b)[:nc]),
+                                           float(wl.bias[b]))
+            got = ids_gpu[b, :int(cnt_gpu[b])].tolist()
+            near = compare_selection(got, ref_ids, z, "%s p%d b%d" % (c.name, p, b))
+            # with near-tie flips, attention is checked over the GPU's own selection
+            use_ids = got if near else ref_ids
+            K, V = wl.seq_kv(b)
+            Kb, Vb = bits(K), bits(V)
+            for s in sorted(keep_steps):
+                ref = oracle.step_output(bits(wl.q(p, s)[b]), Kb, Vb, use_ids, n_ctx, c.W, s,
+                                         c.scale, heads=heads)
+                got_o = outs[(p, s)][b]
+                if heads is not None:
+                    got_o = got_o[list(heads)]
+                compare_attention(got_o, ref, "%s p%d s%d b%d" % (c.name, p, s, b))
+
+
+def test_tiny_every_step(cuda_ok):
+    wl = LI.Workload(LI.tiny(), pin=True)
+    check_loop(wl, set(range(64)))
+
+
+STEPS = {0, 1, 31, 32, 33, 63}
+
+
+@pytest.mark.parametrize("name,cfg", [
+    ("mid_batch_small", lambda: LI.scaled_down(LI.mid_batch(), ctx_blocks=160)),
+    ("long_4pass_small", lambda: LI.scaled_down(LI.long_ctx(), ctx_blocks=200, B=2)),
+    ("ragged_small", lambda: LI.scaled_down(LI.ragged_mix(), ctx_blocks=160, B=12)),
+    ("one_million_geometry_small", lambda: LI.scaled_down(LI.one_million(-1.5), ctx_blocks=300)),
+    ("window_covers_context", lambda: LI.scaled_down(LI.tiny(), ctx_blocks=12, W=1024)),
+])
+def test_scaled_loops(cuda_ok, name, cfg):
+    wl = LI.Workload(cfg(), pin=True)
+    check_loop(wl, STEPS)
+
+
+@pytest.mark.slow
+def test_one_million_full_sampled(cuda_ok):
+    """1,048,576-token context, bias -2: steps 0 and 63 on four sampled heads."""
+    wl = LI.Workload(LI.one_million(-2.0), pin=True)
+    check_loop(wl, {0, 63}, heads=[0, 21, 42, 63])
+
+
+@pytest.mark.slow
+def test_mid_batch_full_sampled(cuda_ok):
+    """B=8 x 131,072 tokens: steps 0 and 63 on two sampled heads of every sequence."""
+    wl = LI.Workload(LI.mid_batch(), pin=True)
+    check_loop(wl, {0, 63}, heads=[5, 60])
