@@ -221,6 +221,16 @@ size_t lsa_state_size(void);
    (set-up before the first lsa_step of a run; not part of the per-step path). */
 lsa_status lsa_load_window(const lsa_state* st, int32_t pass, void* stream);
 
+/* The pieces lsa_step is made of, for callers that schedule or time them separately:
+   lsa_pass_setup  (pass start) candidate counts, resident page lists, zeroed tail pages;
+   lsa_append      (every step) new token into tail slot step % 64, written through to
+                   the host pool; tail_len = step % 64 + 1.
+   lsa_step(step) == [step % 64 == 0: lsa_pass_setup, lsa_index, lsa_gather], lsa_append,
+   lsa_decode_attn, with the state's buffers. */
+lsa_status lsa_pass_setup(const lsa_state* st, int32_t pass, void* stream);
+lsa_status lsa_append(const lsa_state* st, int64_t step, const uint16_t* k_new,
+                      const uint16_t* v_new, void* stream);
+
 /* One decode step. h: device bf16 [L][B][D], read only when step % 64 == 0;
    q: device bf16 [B][H][d]; k_new, v_new: device bf16 [B][d]; out: device bf16 [B][H][d]. */
 lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t* h, const uint16_t* q,

@@ -15,6 +15,7 @@ from . import _lib
 from ._lib import LsaError, LsaState, BLOCK, TAU
 
 __all__ = ["lsa_index", "lsa_gather", "lsa_decode_attn", "lsa_step", "lsa_load_window",
+           "lsa_pass_setup", "lsa_append",
            "index_workspace_size", "decode_attn_workspace_size", "LsaDecoder", "LsaError",
            "LsaState", "BLOCK", "TAU", "library_path"]
 
@@ -112,6 +113,19 @@ def lsa_decode_attn(q, hbm_pool, block_table, n_entries, tail_len, scale: float,
 def lsa_load_window(state: LsaState, pass_idx: int, stream=None) -> None:
     _lib.check("lsa_load_window", _lib.lib().lsa_load_window(C.byref(state), pass_idx,
                                                                _stream(stream)))
+
+
+def lsa_pass_setup(state: LsaState, pass_idx: int, stream=None) -> None:
+    """Pass start bookkeeping of the step driver (lsa_pass_setup in lsa.h)."""
+    _lib.check("lsa_pass_setup", _lib.lib().lsa_pass_setup(C.byref(state), pass_idx,
+                                                             _stream(stream)))
+
+
+def lsa_append(state: LsaState, step: int, k_new, v_new, stream=None) -> None:
+    """Append the step's token to the tail pages (lsa_append in lsa.h)."""
+    st = _lib.lib().lsa_append(C.byref(state), step, _dev(k_new, torch.bfloat16, "k_new"),
+                               _dev(v_new, torch.bfloat16, "v_new"), _stream(stream))
+    _lib.check("lsa_append", st)
 
 
 def lsa_step(state: LsaState, step: int, h, q, k_new, v_new, out, stream=None) -> None:

@@ -62,6 +62,8 @@ SIGNATURES = {
     "lsa_state_size": (_sz, []),
     "lsa_load_window": (_i32, [C.POINTER(LsaState), _i32, _p]),
     "lsa_step": (_i32, [C.POINTER(LsaState), _i64, _p, _p, _p, _p, _p, _p]),
+    "lsa_pass_setup": (_i32, [C.POINTER(LsaState), _i32, _p]),
+    "lsa_append": (_i32, [C.POINTER(LsaState), _i64, _p, _p, _p]),
 }
 
 _lib = None

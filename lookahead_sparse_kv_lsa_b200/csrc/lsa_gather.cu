@@ -302,6 +302,33 @@ extern "C" lsa_status lsa_load_window(const lsa_state* st, int32_t pass, void* s
   return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
 }
 
+extern "C" lsa_status lsa_pass_setup(const lsa_state* st, int32_t pass, void* stream) {
+  const lsa_status v = lsa_state_check(st);
+  if (v != LSA_OK) return v;
+  if (pass < 0) return LSA_ERR_INVALID_ARG;
+  const void* hp = lsa_host::mapped_host_ptr(st->host_pool);
+  if (hp == nullptr) return LSA_ERR_INVALID_ARG;
+  lsa::gth::pass_setup_kernel<<<st->B, lsa::gth::THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+      step_args(st, hp), pass);
+  return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}
+
+extern "C" lsa_status lsa_append(const lsa_state* st, int64_t step, const uint16_t* k_new,
+                                 const uint16_t* v_new, void* stream) {
+  const lsa_status v = lsa_state_check(st);
+  if (v != LSA_OK) return v;
+  if (step < 0 || step / LSA_TAU > (int64_t(1) << 30) || !k_new || !v_new)
+    return LSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15u)
+    return LSA_ERR_INVALID_ARG;
+  const void* hp = lsa_host::mapped_host_ptr(st->host_pool);
+  if (hp == nullptr) return LSA_ERR_INVALID_ARG;
+  lsa::gth::append_kernel<<<st->B, st->d / 8, 0, static_cast<cudaStream_t>(stream)>>>(
+      step_args(st, hp), static_cast<int>(step / LSA_TAU), static_cast<int>(step % LSA_TAU),
+      k_new, v_new);
+  return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}
+
 extern "C" lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t* h,
                                const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
                                uint16_t* out, void* stream) {
@@ -310,19 +337,15 @@ extern "C" lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t
   if (step < 0 || step / LSA_TAU > (int64_t(1) << 30) || !q || !k_new || !v_new || !out)
     return LSA_ERR_INVALID_ARG;
   const int p = static_cast<int>(step / LSA_TAU), s = static_cast<int>(step % LSA_TAU);
-  if (s == 0 && !h) return LSA_ERR_INVALID_ARG;
-  const void* hp = lsa_host::mapped_host_ptr(st->host_pool);
-  if (hp == nullptr) return LSA_ERR_INVALID_ARG;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const lsa::gth::StepArgs a = step_args(st, hp);
-  const int wb1 = a.wb + 1;
   if (s == 0) {
-    lsa::gth::pass_setup_kernel<<<st->B, lsa::gth::THREADS, 0, cs>>>(a, p);
-    if (cudaGetLastError() != cudaSuccess) return LSA_ERR_CUDA;
+    if (!h) return LSA_ERR_INVALID_ARG;
+    v = lsa_pass_setup(st, p, stream);
+    if (v != LSA_OK) return v;
     v = lsa_index(h, st->w_q, st->bias, st->k_idx, st->kidx_off, st->n_cand, st->B, st->L, st->D,
                   st->d_i, st->max_cand, st->sel_ids, st->sel_cnt, st->cap, nullptr, nullptr,
                   st->index_ws, st->index_ws_bytes, st->err, stream);
     if (v != LSA_OK) return v;
+    const int wb1 = st->W / LSA_BLOCK + 1;
     const int64_t base = static_cast<int64_t>(st->B) * wb1;
     v = lsa_gather(st->host_pool, st->host_blocks, st->host_blk_off, st->sel_ids, st->sel_cnt,
                    st->cap, st->res_pages, st->n_res, wb1, st->B, st->d, st->hbm_pool,
@@ -331,8 +354,8 @@ extern "C" lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t
                    st->n_entries, st->err, stream);
     if (v != LSA_OK) return v;
   }
-  lsa::gth::append_kernel<<<st->B, st->d / 8, 0, cs>>>(a, p, s, k_new, v_new);
-  if (cudaGetLastError() != cudaSuccess) return LSA_ERR_CUDA;
+  v = lsa_append(st, step, k_new, v_new, stream);
+  if (v != LSA_OK) return v;
   return lsa_decode_attn(q, st->hbm_pool, st->n_pages, st->block_table, st->bt_stride,
                          st->n_entries, st->tail_len, st->B, st->H, st->d, st->scale, out,
                          st->attn_ws, st->attn_ws_bytes, st->err, stream);

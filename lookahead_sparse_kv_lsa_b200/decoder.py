@@ -89,5 +89,32 @@ class LsaDecoder:
         from . import lsa_step
         lsa_step(self.state, step, h, q, k_new, v_new, out, stream)
 
+    # -- the pieces of one step, as lsa_step composes them ------------------------
+    def pass_setup(self, pass_idx: int, stream=None) -> None:
+        from . import lsa_pass_setup
+        lsa_pass_setup(self.state, pass_idx, stream)
+
+    def index(self, h, stream=None) -> None:
+        from . import lsa_index
+        lsa_index(h, self.w_q, self.bias, self.k_idx, self.kidx_off, self.n_cand, self.max_cand,
+                  self.sel_ids if self.cap > 0 else self.sel_ids[:, :0], self.sel_cnt,
+                  self.index_ws, self.err, stream=stream)
+
+    def gather(self, stream=None) -> None:
+        from . import lsa_gather
+        base = self.B * (self.W // BLOCK + 1)
+        lsa_gather(self.host_pool, self.host_blk_off, self.sel_ids, self.sel_cnt, self.res_pages,
+                   self.n_res, self.hbm_pool, base, self.n_pages - base, self.block_table,
+                   self.n_entries, self.err, stream)
+
+    def append(self, step: int, k_new, v_new, stream=None) -> None:
+        from . import lsa_append
+        lsa_append(self.state, step, k_new, v_new, stream)
+
+    def attend(self, q, out, stream=None) -> None:
+        from . import lsa_decode_attn
+        lsa_decode_attn(q, self.hbm_pool, self.block_table, self.n_entries, self.tail_len,
+                        self.state.scale, out, self.attn_ws, self.err, stream)
+
     def read_err(self) -> int:
         return int(self.err.item())
