@@ -41,6 +41,7 @@ DEFAULT_WORKLOAD = "1m_b20"
 FALLBACK_HBM_GBS = 6650.0
 LAUNCHES_PER_DECODE_STEP = 3      # append, split-K attention, merge
 LAUNCHES_PER_PASS_HEAD = 4        # pass set-up, projection, scoring, gather
+SEL_PAGES = 4096                  # HBM pages for kept blocks (1,079 used at bias -2; 512 MB)
 
 
 def parse_args():
@@ -186,7 +187,8 @@ def make_decoder(wl, dev):
     max_cand = max(1, max(n_cand))
     dec = lsa.LsaDecoder(wl.w_q.to(dev), wl.k_idx.to(dev), wl.blk_off[:c.B],
                          torch.from_numpy(wl.bias).to(dev), wl.host_pool, wl.blk_off, wl.nb0,
-                         W=c.W, H=c.H, cap=max_cand, max_cand=max_cand, scale=c.scale)
+                         W=c.W, H=c.H, cap=max_cand, max_cand=max_cand, scale=c.scale,
+                         sel_pages=min(c.B * max_cand, SEL_PAGES))
     dec.load_window(0)
     return dec, n_cand
 

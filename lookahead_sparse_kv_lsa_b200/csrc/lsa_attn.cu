@@ -574,14 +574,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // Log-sum-exp merge of the partial results of every segment of sequence b, head h:
 //   M = max_k m_k,  out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k   (m in log2 units)
 // The segments of b are the CTAs whose unit ranges meet b's units; slot = CTA + b.
-// grid (H, B), d/4 threads, each owning 4 consecutive dimensions.
-__global__ void __launch_bounds__(128) attn_merge_kernel(const Args a, int G, uint16_t* out) {
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  __shared__ long long s_tot[2];
-  __shared__ long long s_part[4][2];
+// grid (H, B, d/128), MERGE_THREADS threads: the split weights are computed once per
+// block into shared memory, then the warps split the partials among themselves (each
+// lane owning 4 consecutive dimensions) and are summed through shared memory.
+constexpr int MERGE_THREADS = 256;
+constexpr int MERGE_WARPS = MERGE_THREADS / 32;
+
+__global__ void __launch_bounds__(MERGE_THREADS) attn_merge_kernel(const Args a, int G,
+                                                                   uint16_t* out) {
+  extern __shared__ float s_w[];          // [G] split weights
+  __shared__ long long s_part[MERGE_WARPS][2];
+  __shared__ float s_red[MERGE_WARPS];
+  __shared__ float4 s_acc[MERGE_WARPS][32];
+  const int h = blockIdx.x, b = blockIdx.y, dchunk = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // prefix of units before b, and the batch total
   long long before = 0, total = 0;
-  for (int i = tid; i < a.B; i += blockDim.x) {
+  for (int i = tid; i < a.B; i += MERGE_THREADS) {
     const int u = seq_units(a, i);
     total += u;
     if (i < b) before += u;
@@ -591,59 +600,93 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const Args a, int G, ui
     total += __shfl_xor_sync(0xffffffffu, total, o);
     before += __shfl_xor_sync(0xffffffffu, before, o);
   }
-  if ((tid & 31) == 0) {
-    s_part[tid >> 5][0] = total;
-    s_part[tid >> 5][1] = before;
+  if (lane == 0) {
+    s_part[warp][0] = total;
+    s_part[warp][1] = before;
   }
   __syncthreads();
-  if (tid == 0) {
-    long long t = 0, bf = 0;
-    for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) {
-      t += s_part[w][0];
-      bf += s_part[w][1];
-    }
-    s_tot[0] = t;
-    s_tot[1] = bf;
-    if (h == 0 && seq_malformed(a, b)) set_err(a.err, LSA_DEVERR_BAD_SIZE);
+  long long U = 0, P = 0;
+#pragma unroll
+  for (int w = 0; w < MERGE_WARPS; ++w) {
+    U += s_part[w][0];
+    P += s_part[w][1];
   }
-  __syncthreads();
-  const long long U = s_tot[0], P = s_tot[1];
+  if (tid == 0 && h == 0 && dchunk == 0 && seq_malformed(a, b)) set_err(a.err, LSA_DEVERR_BAD_SIZE);
   const int ub = seq_units(a, b);
-  const int d0 = tid * 4;
+  const int d0 = dchunk * 128 + lane * 4;
   uint16_t* dst = out + (static_cast<long long>(b) * a.H + h) * a.d + d0;
-  if (d0 >= a.d) return;
   if (ub == 0) {
-    *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+    if (warp == 0) *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
     return;
   }
-  // CTA holding unit u: the largest c with floor(c*U/G) <= u
+  // CTA holding unit u: the largest c with floor(c*U/G) <= u; CTAs whose unit range is
+  // empty (grid larger than the work) hold no slot
   const long long c_lo = ((P + 1) * G - 1) / U;
   const long long c_hi = ((P + ub) * G - 1) / U;
-  // CTAs with an empty unit range (when the grid outnumbers the units) hold no slot
-  auto empty_cta = [&](long long c) { return (c * U) / G == ((c + 1) * U) / G; };
-  float M = -INFINITY;
-  for (long long c = c_lo; c <= c_hi; ++c)
-    if (!empty_cta(c)) M = fmaxf(M, a.part_ml[((c + b) * a.H + h) * 2]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int n = static_cast<int>(c_hi - c_lo + 1);
+  float mx = -INFINITY;
+  for (int k = tid; k < n; k += MERGE_THREADS) {
+    const long long c = c_lo + k;
+    float m = -INFINITY;
+    if ((c * U) / G != ((c + 1) * U) / G) m = a.part_ml[((c + b) * a.H + h) * 2];
+    s_w[k] = m;
+    mx = fmaxf(mx, m);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) s_red[warp] = mx;
+  __syncthreads();
+  float M = s_red[0];
+#pragma unroll
+  for (int w = 1; w < MERGE_WARPS; ++w) M = fmaxf(M, s_red[w]);
+  __syncthreads();
+  float ls = 0.f;
+  for (int k = tid; k < n; k += MERGE_THREADS) {
+    const long long c = c_lo + k;
+    const float m = s_w[k];
+    const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+    if (w != 0.f) ls += w * a.part_ml[((c + b) * a.H + h) * 2 + 1];
+    s_w[k] = w;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  if (lane == 0) s_red[warp] = ls;
+  __syncthreads();
   float lsum = 0.f;
-  for (long long c = c_lo; c <= c_hi; ++c) {
-    if (empty_cta(c)) continue;
-    const long long slot = c + b;
-    const float w = exp2f(a.part_ml[(slot * a.H + h) * 2] - M);
-    lsum += w * a.part_ml[(slot * a.H + h) * 2 + 1];
-    const float4 o = *reinterpret_cast<const float4*>(a.part_o + (slot * a.H + h) * a.d + d0);
+#pragma unroll
+  for (int w = 0; w < MERGE_WARPS; ++w) lsum += s_red[w];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int k = warp; k < n; k += MERGE_WARPS) {
+    const float w = s_w[k];
+    if (w == 0.f) continue;
+    const long long slot = c_lo + k + b;
+    const float4 o = __ldcg(reinterpret_cast<const float4*>(a.part_o + (slot * a.H + h) * a.d + d0));
     acc.x += w * o.x;
     acc.y += w * o.y;
     acc.z += w * o.z;
     acc.w += w * o.w;
   }
-  const float inv = 1.f / lsum;
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-  uint2 pk;
-  pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-  pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(dst) = pk;
+  s_acc[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float4 t = s_acc[0][lane];
+#pragma unroll
+    for (int w = 1; w < MERGE_WARPS; ++w) {
+      const float4 v = s_acc[w][lane];
+      t.x += v.x;
+      t.y += v.y;
+      t.z += v.z;
+      t.w += v.w;
+    }
+    const float inv = 1.f / lsum;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(t.x * inv, t.y * inv);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(t.z * inv, t.w * inv);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(dst) = pk;
+  }
 }
 
 }  // namespace attn
@@ -748,6 +791,7 @@ extern "C" lsa_status lsa_decode_attn(const uint16_t* q, const uint16_t* hbm_poo
     default: st = dispatch_d<64>(mkv, mq, a, G, s); break;
   }
   if (st != LSA_OK) return st;
-  lsa::attn::attn_merge_kernel<<<dim3(H, B), d / 4, 0, s>>>(a, G, out);
+  lsa::attn::attn_merge_kernel<<<dim3(H, B, d / 128), lsa::attn::MERGE_THREADS,
+                                 G * sizeof(float), s>>>(a, G, out);
   return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
 }
