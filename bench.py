@@ -39,7 +39,7 @@ METRIC = "LSA decode tokens/s (index+gather+sparse attn) at 1M ctx; attn HBM GB/
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "1m_b20"
 FALLBACK_HBM_GBS = 6650.0
-LAUNCHES_PER_DECODE_STEP = 3      # append, split-K attention, merge
+LAUNCHES_PER_DECODE_STEP = 1      # one fused kernel: append + split-K attention + merge
 LAUNCHES_PER_PASS_HEAD = 4        # pass set-up, projection, scoring, gather
 SEL_PAGES = 4096                  # HBM pages for kept blocks (1,079 used at bias -2; 512 MB)
 
@@ -194,7 +194,8 @@ def make_decoder(wl, dev):
 
 
 def run_pass(dec, inp, out, evs=None):
-    """One pass through the library's public calls, as lsa_step composes them."""
+    """One pass through the library's public calls, exactly as lsa_step composes them:
+    lsa_pass_setup, lsa_index, lsa_gather, then lsa_decode_step for each decode step."""
     dec.pass_setup(0)
     if evs is not None:
         evs[0].record()
@@ -205,12 +206,9 @@ def run_pass(dec, inp, out, evs=None):
     if evs is not None:
         evs[2].record()
     for s in range(inp.q.shape[0]):
-        dec.append(s, inp.k[s], inp.v[s])
+        dec.decode_step(s, inp.q[s], inp.k[s], inp.v[s], out[s])
         if evs is not None:
-            evs[3 + 2 * s].record()
-        dec.attend(inp.q[s], out[s])
-        if evs is not None:
-            evs[4 + 2 * s].record()
+            evs[3 + s].record()
 
 
 def capture(dec, inp, out, n_steps):
@@ -219,7 +217,7 @@ def capture(dec, inp, out, n_steps):
     stream = torch.cuda.Stream()
     for _ in range(n_steps):
         evs = [torch.cuda.Event(enable_timing=True, external=True)
-               for _ in range(3 + 2 * inp.q.shape[0])]
+               for _ in range(3 + inp.q.shape[0])]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
             run_pass(dec, inp, out, evs)
@@ -231,9 +229,8 @@ def capture(dec, inp, out, n_steps):
 def event_breakdown(evs, tau):
     idx = evs[0].elapsed_time(evs[1])
     gth = evs[1].elapsed_time(evs[2])
-    attn = [evs[3 + 2 * s].elapsed_time(evs[4 + 2 * s]) for s in range(tau)]
-    app = [evs[2 + 2 * s].elapsed_time(evs[3 + 2 * s]) for s in range(tau)]
-    return idx, gth, attn, app
+    step = [evs[2 + s].elapsed_time(evs[3 + s]) for s in range(tau)]
+    return idx, gth, step
 
 
 def attn_bytes_per_step(cfg, n_sel, s):
@@ -341,7 +338,7 @@ def oracle_pass_seconds(wl, steps):
     return t_idx + c.tau * per_step, time.perf_counter() - t_start
 
 
-def cpu_baseline(wl, steps=(0, 31, 63)):
+def cpu_baseline(wl, steps=tuple(range(0, 64, 3))):
     c = wl.cfg
     t_pass, spent = oracle_pass_seconds(wl, steps)
     return {"value": c.B * c.tau / t_pass, "unit": UNIT, "cores": oracle_threads(),
@@ -508,15 +505,15 @@ def run_lsa(args, rank, world, local):
         raise SystemExit("device error word %d in the timed region" % dec.read_err())
 
     # per-call durations from the events inside the graphs (their last, timed, replay)
-    idx_ms, gth_ms, attn_ms, app_ms = [], [], [], []
+    idx_ms, gth_ms, attn_ms = [], [], []
     for i in range(n_graphs):
-        a, g, at, ap = event_breakdown(events[i], cfg.tau)
-        idx_ms.append(a); gth_ms.append(g); attn_ms += at; app_ms += ap
+        a, g, at = event_breakdown(events[i], cfg.tau)
+        idx_ms.append(a); gth_ms.append(g); attn_ms += at
     hbm, peak_src = peaks()
     attn_bytes = sum(attn_bytes_per_step(cfg, n_sel, s) for s in range(cfg.tau)) / cfg.tau
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
-    traffic, traffic_src = profiled_traffic("attn_splitk_1m_b20")
+    traffic, traffic_src = profiled_traffic("attn_decode_step_1m_b20")
     ib = index_bytes(cfg, n_cand, n_sel)
     idx_avg = statistics.mean(idx_ms)
     gather_bytes = sum(n_sel) * 2 * 64 * cfg.d * 2
@@ -535,7 +532,8 @@ def run_lsa(args, rank, world, local):
                    "l2": "inputs larger than L2: each decode step streams %.0f MB of attended KV"
                          % (attn_bytes / 1e6),
                    "launch": "one CUDA graph per step"},
-        "roofline": {"bound": "hbm", "kernel": "lsa_decode_attn (split-K attention + LSE merge)",
+        "roofline": {"bound": "hbm",
+                     "kernel": "lsa_decode_step (fused append + split-K attention + LSE merge)",
                      "achieved": achieved, "peak": hbm, "peak_source": peak_src,
                      "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": traffic, "traffic_source": traffic_src,
@@ -549,7 +547,6 @@ def run_lsa(args, rank, world, local):
                    "achieved_GBs": gather_bytes / (gth_avg * 1e-3) / 1e9,
                    "pinned_h2d_GBs": h2d_peak,
                    "frac": gather_bytes / (gth_avg * 1e-3) / 1e9 / h2d_peak},
-        "append_avg_ms": statistics.mean(app_ms),
         "gpu_launches": args.steps * (LAUNCHES_PER_PASS_HEAD + cfg.tau * LAUNCHES_PER_DECODE_STEP),
         "clocks": clocks,
     }

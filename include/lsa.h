@@ -172,10 +172,13 @@ size_t lsa_decode_attn_workspace_size(int32_t B, int32_t H, int32_t d, int32_t n
  * rings (block j of sequence b lives in page b*(wb+1) + j % (wb+1)); pages
  * [B*(wb+1), n_pages) receive the kept blocks of the current pass.
  *
- *   step % 64 == 0: pass set-up kernel (n_cand, resident page lists, zero the new
- *                   tail page), lsa_index on h, lsa_gather of the kept blocks;
- *   every step:     append k_new / v_new at slot step % 64 of each tail page (written
- *                   through to the host pool), then lsa_decode_attn into out.
+ *   step % 64 == 0: pass set-up kernel (n_cand, resident page lists, write-back of the
+ *                   previous tail page to the host pool, zero the new tail page),
+ *                   lsa_index on h, lsa_gather of the kept blocks;
+ *   every step:     append k_new / v_new at slot step % 64 of each tail page, fused into
+ *                   the decode-attention kernel, which writes out.
+ * The tail page of the last pass of a run reaches the host pool only when a following
+ * pass starts; the window keeps it resident in HBM meanwhile.
  *
  * All pointers in lsa_state are owned by the caller; the struct is plain data.
  */
@@ -222,12 +225,20 @@ size_t lsa_state_size(void);
 lsa_status lsa_load_window(const lsa_state* st, int32_t pass, void* stream);
 
 /* The pieces lsa_step is made of, for callers that schedule or time them separately:
-   lsa_pass_setup  (pass start) candidate counts, resident page lists, zeroed tail pages;
-   lsa_append      (every step) new token into tail slot step % 64, written through to
-                   the host pool; tail_len = step % 64 + 1.
-   lsa_step(step) == [step % 64 == 0: lsa_pass_setup, lsa_index, lsa_gather], lsa_append,
-   lsa_decode_attn, with the state's buffers. */
+   lsa_pass_setup  (pass start) candidate counts, resident page lists, a zeroed new tail
+                   page; from pass 1 on it also writes the previous pass's completed tail
+                   page back to the host pool;
+   lsa_decode_step (every step) lsa_decode_attn with the token append fused into it: the
+                   CTA that reads a sequence's tail page first stores k_new / v_new into
+                   slot step % 64 of it; tail_len = step % 64 + 1.
+   lsa_step(step) == [step % 64 == 0: lsa_pass_setup, lsa_index, lsa_gather],
+                     lsa_decode_step, with the state's buffers.
+   lsa_append is the stand-alone append (HBM tail page and host pool), for callers that
+   run lsa_decode_attn themselves. */
 lsa_status lsa_pass_setup(const lsa_state* st, int32_t pass, void* stream);
+lsa_status lsa_decode_step(const lsa_state* st, int64_t step, const uint16_t* q,
+                           const uint16_t* k_new, const uint16_t* v_new, uint16_t* out,
+                           void* stream);
 lsa_status lsa_append(const lsa_state* st, int64_t step, const uint16_t* k_new,
                       const uint16_t* v_new, void* stream);
 

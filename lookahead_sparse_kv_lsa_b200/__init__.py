@@ -15,7 +15,7 @@ from . import _lib
 from ._lib import LsaError, LsaState, BLOCK, TAU
 
 __all__ = ["lsa_index", "lsa_gather", "lsa_decode_attn", "lsa_step", "lsa_load_window",
-           "lsa_pass_setup", "lsa_append",
+           "lsa_pass_setup", "lsa_append", "lsa_decode_step",
            "index_workspace_size", "decode_attn_workspace_size", "LsaDecoder", "LsaError",
            "LsaState", "BLOCK", "TAU", "library_path"]
 
@@ -126,6 +126,15 @@ def lsa_append(state: LsaState, step: int, k_new, v_new, stream=None) -> None:
     st = _lib.lib().lsa_append(C.byref(state), step, _dev(k_new, torch.bfloat16, "k_new"),
                                _dev(v_new, torch.bfloat16, "v_new"), _stream(stream))
     _lib.check("lsa_append", st)
+
+
+def lsa_decode_step(state: LsaState, step: int, q, k_new, v_new, out, stream=None) -> None:
+    """Decode attention with the token append fused in (lsa_decode_step in lsa.h)."""
+    st = _lib.lib().lsa_decode_step(C.byref(state), step, _dev(q, torch.bfloat16, "q"),
+                                    _dev(k_new, torch.bfloat16, "k_new"),
+                                    _dev(v_new, torch.bfloat16, "v_new"),
+                                    _dev(out, torch.bfloat16, "out"), _stream(stream))
+    _lib.check("lsa_decode_step", st)
 
 
 def lsa_step(state: LsaState, step: int, h, q, k_new, v_new, out, stream=None) -> None:

@@ -64,6 +64,7 @@ SIGNATURES = {
     "lsa_step": (_i32, [C.POINTER(LsaState), _i64, _p, _p, _p, _p, _p, _p]),
     "lsa_pass_setup": (_i32, [C.POINTER(LsaState), _i32, _p]),
     "lsa_append": (_i32, [C.POINTER(LsaState), _i64, _p, _p, _p]),
+    "lsa_decode_step": (_i32, [C.POINTER(LsaState), _i64, _p, _p, _p, _p, _p]),
 }
 
 _lib = None

@@ -38,6 +38,8 @@ constexpr int STAGE_BYTES = TILE * 128;   // [128 rows][64 bf16] = 16 KB
 constexpr int NTHREADS = 192;
 constexpr int MAXSEG = 16;                // segments planned per batch
 constexpr float RESCALE_LOG2 = 8.0f;      // raise the running max only by more than 2^8
+constexpr int MAXITEMS = 32;              // merge items (sequence, head) per CTA and round
+constexpr int MAX_GRID = 256;             // CTAs per launch (one per SM)
 
 struct Seg {
   int b, u0, u1;
@@ -46,7 +48,7 @@ struct Seg {
 struct Misc {
   uint64_t full[NST], empty[NST];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, q_full, q_free, mma_done;
+  uint64_t p_full, pv_done, q_full, q_free, mma_done, merge_bar;
   uint32_t tmem_base;
   int abort;
   int nseg, more;
@@ -54,34 +56,48 @@ struct Misc {
   float red[4][64];
   float m_use[64];
   float alpha[64];
+  // fused merge
+  int n_items, total_items;
+  int item_b[MAXITEMS], item_h[MAXITEMS], item_clo[MAXITEMS], item_chi[MAXITEMS];
+  float wgt[MAX_GRID];
 };
 
 struct Args {
   const int32_t* block_table;
   const int32_t* n_entries;
   const int32_t* tail_len;
-  float* part_o;    // [slots][H][d] fp32
-  float* part_ml;   // [slots][H][2] fp32 (running max in log2 units, denominator)
+  float* part_o;          // [slots][H][d] fp32
+  float* part_ml;         // [slots][H][2] fp32 (running max in log2 units, denominator)
+  unsigned int* sync;     // [2] grid-barrier arrive / depart counters (left at zero)
+  uint16_t* out;          // [B][H][d] bf16
+  uint16_t* pool;         // the HBM pool (written only by the fused append)
+  const uint16_t* k_new;  // fused append: [B][d] token written into slot fused_tail-1
+  const uint16_t* v_new;  //   of each tail page (nullptr: no append)
+  int32_t* tail_len_out;  // fused append: receives fused_tail per sequence (nullable)
   int32_t* err;
   long long n_pages;
   int bt_stride, B, H, d;
+  int fused_tail;         // > 0: every sequence's tail length (tail_len is not read)
   float scale_log2;
 };
 
 // Units (32-token pieces) of sequence b; 0 for an empty or malformed sequence.
+__device__ __forceinline__ int seq_tail(const Args& a, int b) {
+  return a.fused_tail > 0 ? a.fused_tail : __ldg(a.tail_len + b);
+}
+
 __device__ __forceinline__ int seq_units(const Args& a, int b) {
   const int n = __ldg(a.n_entries + b);
-  if (n <= 0) return 0;
-  const int t = __ldg(a.tail_len + b);
-  if (n > a.bt_stride || t < 1 || t > 64) return 0;
+  const int t = seq_tail(a, b);
+  if (n <= 0 || n > a.bt_stride || t < 1 || t > 64) return 0;
   return 2 * (n - 1) + (t + UNIT - 1) / UNIT;
 }
 
 __device__ __forceinline__ bool seq_malformed(const Args& a, int b) {
   const int n = __ldg(a.n_entries + b);
+  const int t = seq_tail(a, b);
   if (n < 0) return true;
   if (n == 0) return false;
-  const int t = __ldg(a.tail_len + b);
   return n > a.bt_stride || t < 1 || t > 64;
 }
 
@@ -96,7 +112,7 @@ __device__ __forceinline__ long long warp_total_units(const Args& a, int lane) {
 
 // Warp 0: list the segments of units [us, ue), skipping the first `skip` of them; at most
 // MAXSEG are stored. Sets m->more when segments remain after the stored ones.
-__device__ void plan_segments(const Args& a, long long us, long long ue, int skip, Misc* m,
+__device__ __noinline__ void plan_segments(const Args& a, long long us, long long ue, int skip, Misc* m,
                               int lane) {
   int found = 0, stored = 0;
   bool more = false;
@@ -182,6 +198,216 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[HP]) {
   for (int c = 0; c < HP / 16; ++c) tmem_ld16(taddr + 16 * c, v + 16 * c);
 }
 
+// CTA holding unit u of the grid-wide split: the largest c with floor(c*U/G) <= u.
+__device__ __forceinline__ long long cta_of_unit(long long u, long long U, long long G) {
+  return ((u + 1) * G - 1) / U;
+}
+__device__ __forceinline__ bool cta_empty(long long c, long long U, long long G) {
+  return (c * U) / G == ((c + 1) * U) / G;
+}
+
+// Warp 0: list this CTA's merge items for round `round`. Items are the (sequence, head)
+// pairs of every sequence whose units span more than one CTA, numbered in sequence
+// order; item j belongs to CTA j % G. Returns the batch's item total (all lanes).
+__device__ __noinline__ int plan_merge(const Args& a, long long U, int round, Misc* m, int lane) {
+  const long long G = gridDim.x;
+  const int cta = blockIdx.x;
+  long long base_u = 0;
+  int base_item = 0, mine = 0;
+  for (int b0 = 0; b0 < a.B; b0 += 32) {
+    const int b = b0 + lane;
+    const int u = b < a.B ? seq_units(a, b) : 0;
+    long long incl = u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const long long p = base_u + incl - u;
+    long long clo = 0, chi = 0;
+    bool split = false;
+    if (u > 0) {
+      clo = cta_of_unit(p, U, G);
+      chi = cta_of_unit(p + u - 1, U, G);
+      split = clo != chi;
+    }
+    const int items = split ? a.H : 0;
+    int iincl = items;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, iincl, o);
+      if (lane >= o) iincl += t;
+    }
+    const int ibase = base_item + iincl - items;
+    if (items > 0) {
+      // first item of this sequence owned by this CTA, then every G-th
+      int j = ibase + static_cast<int>(((cta - ibase) % G + G) % G);
+      for (; j < ibase + items; j += static_cast<int>(G)) {
+        const int rank = (j - cta) / static_cast<int>(G) - round * MAXITEMS;
+        if (rank >= 0 && rank < MAXITEMS) {
+          m->item_b[rank] = b;
+          m->item_h[rank] = j - ibase;
+          m->item_clo[rank] = static_cast<int>(clo);
+          m->item_chi[rank] = static_cast<int>(chi);
+        }
+      }
+    }
+    base_u += __shfl_sync(0xffffffffu, incl, 31);
+    base_item += __shfl_sync(0xffffffffu, iincl, 31);
+  }
+  // items of this CTA: those j < base_item with j % G == cta
+  const int total = base_item;
+  if (total > cta) mine = (total - cta + static_cast<int>(G) - 1) / static_cast<int>(G);
+  if (lane == 0) {
+    m->total_items = total;
+    const int left = mine - round * MAXITEMS;
+    m->n_items = left < 0 ? 0 : (left > MAXITEMS ? MAXITEMS : left);
+  }
+  return total;
+}
+
+// Block-wide reductions over the CTA's threads through m->red[0][*].
+__device__ __forceinline__ float block_max(float v, Misc* m, int tid, int nwarps) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if ((tid & 31) == 0) m->red[0][tid >> 5] = v;
+  __syncthreads();
+  float r = m->red[0][0];
+  for (int w = 1; w < nwarps; ++w) r = fmaxf(r, m->red[0][w]);
+  return r;
+}
+__device__ __forceinline__ float block_sum(float v, Misc* m, int tid, int nwarps) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if ((tid & 31) == 0) m->red[0][tid >> 5] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int w = 0; w < nwarps; ++w) r += m->red[0][w];
+  return r;
+}
+
+// Fused log-sum-exp merge, run by every thread of every CTA after its segments:
+//   M = max_k m_k,  out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k   (m in log2 units)
+// over the partials k of a split sequence. A grid-wide barrier (one arrival counter,
+// bounded wait) separates the partial writes from the reads; the partial rows of one
+// (sequence, head) item are brought into shared memory with 1-D bulk copies, then
+// every thread reduces a slice of the head dimension over all partials.
+__device__ __noinline__ void merge_phase(const Args& a, Misc* m, uint8_t* buf, int buf_bytes, long long U,
+                            bool aborted, uint32_t& merge_phase_bit) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthr = blockDim.x, nwarps = nthr >> 5;
+  const long long G = gridDim.x;
+  volatile int* abort = &m->abort;
+  if (warp == 0) plan_merge(a, U, 0, m, lane);
+  __syncthreads();
+  const int total = m->total_items;
+  if (total == 0) return;             // nothing split: no barrier, every CTA agrees
+  // ---- grid barrier: all partials written before any is read
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(a.sync, 1u);
+    const uint64_t t0 = globaltimer_ns();
+    bool ok = true;
+    while (ld_acquire_gpu(a.sync) < static_cast<unsigned int>(G)) {
+      if (globaltimer_ns() - t0 > LSA_WAIT_LIMIT_NS) {
+        ok = false;
+        break;
+      }
+    }
+    __threadfence();
+    fence_proxy_async_global();       // the partials are read back by bulk copies
+    if (!ok) {
+      set_err(a.err, LSA_DEVERR_TIMEOUT);
+      *abort = 1;
+    }
+  }
+  __syncthreads();
+  bool failed = *abort != 0 || aborted;   // the same value in every thread
+  if (!failed) {
+    float* fbuf = reinterpret_cast<float*>(buf);
+    for (int round = 0;; ++round) {
+      if (round > 0) {
+        __syncthreads();
+        if (warp == 0) plan_merge(a, U, round, m, lane);
+        __syncthreads();
+      }
+      const int n_items = m->n_items;
+      if (n_items == 0) break;
+      for (int it = 0; it < n_items && !failed; ++it) {
+        const int b = m->item_b[it], h = m->item_h[it];
+        const int clo = m->item_clo[it], n = m->item_chi[it] - clo + 1;
+        // split weights
+        float mx = -INFINITY;
+        for (int k = tid; k < n; k += nthr) {
+          const long long c = clo + k;
+          const float mk =
+              cta_empty(c, U, G) ? -INFINITY : __ldcg(a.part_ml + ((c + b) * a.H + h) * 2);
+          m->wgt[k] = mk;
+          mx = fmaxf(mx, mk);
+        }
+        const float M = block_max(mx, m, tid, nwarps);
+        float ls = 0.f;
+        for (int k = tid; k < n; k += nthr) {
+          const long long c = clo + k;
+          const float mk = m->wgt[k];
+          const float w = mk == -INFINITY ? 0.f : exp2f(mk - M);
+          if (w != 0.f) ls += w * __ldcg(a.part_ml + ((c + b) * a.H + h) * 2 + 1);
+          m->wgt[k] = w;
+        }
+        const float inv_l = 1.f / block_sum(ls, m, tid, nwarps);
+        // partial rows, in chunks of the head dimension that fit the buffer
+        int chunk = (buf_bytes / (n * 4)) / 32 * 32;
+        if (chunk > a.d) chunk = a.d;
+        for (int d0 = 0; d0 < a.d && !failed; d0 += chunk) {
+          const int cw = min(chunk, a.d - d0);
+          if (tid == 0) {
+            fence_proxy_async_smem();     // earlier generic accesses of the buffer first
+            uint32_t bytes = 0;
+            for (int k = 0; k < n; ++k)
+              if (m->wgt[k] != 0.f) bytes += cw * 4;
+            mbar_arrive_expect_tx(&m->merge_bar, bytes);
+            for (int k = 0; k < n; ++k) {
+              if (m->wgt[k] == 0.f) continue;
+              const long long slot = clo + k + b;
+              bulk_load(fbuf + static_cast<long long>(k) * cw,
+                        a.part_o + (slot * a.H + h) * a.d + d0, cw * 4, &m->merge_bar);
+            }
+          }
+          const bool ok = __syncthreads_and(mbar_wait(&m->merge_bar, merge_phase_bit, nullptr)) != 0;
+          merge_phase_bit ^= 1u;
+          if (!ok) {
+            failed = true;
+            if (tid == 0) set_err(a.err, LSA_DEVERR_TIMEOUT);
+          } else {
+            uint16_t* dst = a.out + (static_cast<long long>(b) * a.H + h) * a.d + d0;
+            for (int j = tid; j < cw; j += nthr) {
+              float acc = 0.f;
+              for (int k = 0; k < n; ++k) {
+                const float w = m->wgt[k];
+                if (w != 0.f) acc += w * fbuf[static_cast<long long>(k) * cw + j];
+              }
+              const __nv_bfloat16 v = __float2bfloat16_rn(acc * inv_l);
+              dst[j] = *reinterpret_cast<const uint16_t*>(&v);
+            }
+          }
+          __syncthreads();  // the buffer is refilled by the next chunk
+        }
+      }
+      if (failed || m->n_items < MAXITEMS) break;
+    }
+  }
+  // ---- departure: the last CTA out resets the counters for the next launch
+  __syncthreads();
+  if (tid == 0) {
+    if (atomicAdd(a.sync + 1, 1u) == static_cast<unsigned int>(G) - 1u) {
+      atomicExch(a.sync, 0u);
+      atomicExch(a.sync + 1, 0u);
+    }
+  }
+}
+
 template <int HP, int NDC>
 struct Layout {
   static constexpr int NDB = NDC / 2;                   // 128-dim blocks of O^T
@@ -232,6 +458,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&m->q_full, 1);
     mbar_init(&m->q_free, 1);
     mbar_init(&m->mma_done, 1);
+    mbar_init(&m->merge_bar, 1);
     m->abort = 0;
     fence_barrier_init();
   }
@@ -267,6 +494,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   for (int batch = 0;; ++batch) {
     const int nseg = m->nseg;
+    if (warp == 0 && a.k_new != nullptr) {
+      // Fused append: the CTA that owns a sequence's last unit writes the step's token
+      // into its tail page before this warp's TMA loads read that page.
+      for (int g = 0; g < nseg; ++g) {
+        const Seg sg = m->seg[g];
+        if (sg.u1 != seq_units(a, sg.b)) continue;
+        const int n = __ldg(a.n_entries + sg.b);
+        const int page = __ldg(a.block_table + static_cast<long long>(sg.b) * a.bt_stride + n - 1);
+        if (page < 0 || page >= a.n_pages) continue;  // reported by the producer
+        const long long row = static_cast<long long>(page) * 128 + (a.fused_tail - 1);
+        const uint4* ks = reinterpret_cast<const uint4*>(a.k_new + static_cast<long long>(sg.b) * a.d);
+        const uint4* vs = reinterpret_cast<const uint4*>(a.v_new + static_cast<long long>(sg.b) * a.d);
+        uint4* kd = reinterpret_cast<uint4*>(a.pool + row * a.d);
+        uint4* vd = reinterpret_cast<uint4*>(a.pool + (row + 64) * a.d);
+        for (int i = lane; i < a.d / 8; i += 32) {
+          kd[i] = __ldg(ks + i);
+          vd[i] = __ldg(vs + i);
+        }
+        if (lane == 0 && a.tail_len_out != nullptr) a.tail_len_out[sg.b] = a.fused_tail;
+      }
+      fence_proxy_async_global();
+      __syncwarp();
+    }
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
@@ -404,7 +654,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const Seg sg = m->seg[g];
         const int T = (sg.u1 - sg.u0 + 3) >> 2;
         const int n_ent = __ldg(a.n_entries + sg.b);
-        const int tl = __ldg(a.tail_len + sg.b);
+        const int tl = seq_tail(a, sg.b);
         float m_run = -INFINITY;               // running max (log2 units) of head t128
         float lp[HP];
 #pragma unroll
@@ -513,14 +763,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           failed = true;
           break;
         }
+        // a sequence held whole by this CTA is normalised and written out here; a split
+        // one leaves its partial (O, m, l) in slot CTA + sequence for the merge
+        const bool whole = sg.u0 == 0 && sg.u1 == seq_units(a, sg.b);
         const long long slot = static_cast<long long>(blockIdx.x) + sg.b;
         if (t128 < a.H) {
           const int h = t128;
           const float l = m->red[0][h] + m->red[1][h] + m->red[2][h] + m->red[3][h];
-          a.part_ml[(slot * a.H + h) * 2 + 0] = m_run;
-          a.part_ml[(slot * a.H + h) * 2 + 1] = l;
+          if (whole) {
+            m->alpha[h] = 1.f / l;
+          } else {
+            a.part_ml[(slot * a.H + h) * 2 + 0] = m_run;
+            a.part_ml[(slot * a.H + h) * 2 + 1] = l;
+          }
         }
+        if (whole) named_bar_sync(1, 128);
         float* po = a.part_o + slot * a.H * a.d;
+        uint16_t* fo = a.out + static_cast<long long>(sg.b) * a.H * a.d;
 #pragma unroll
         for (int db = 0; db < NDB; ++db) {
 #pragma unroll
@@ -531,7 +790,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int h = 16 * c + i;
-              if (h < a.H) po[static_cast<long long>(h) * a.d + db * 128 + row] = o[i];
+              if (h < a.H) {
+                const long long idx = static_cast<long long>(h) * a.d + db * 128 + row;
+                if (whole) {
+                  const __nv_bfloat16 v = __float2bfloat16_rn(o[i] * m->alpha[h]);
+                  fo[idx] = *reinterpret_cast<const uint16_t*>(&v);
+                } else {
+                  po[idx] = o[i];
+                }
+              }
             }
           }
         }
@@ -569,123 +836,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, LY::TMEM_COLS);
-}
-
-// Log-sum-exp merge of the partial results of every segment of sequence b, head h:
-//   M = max_k m_k,  out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k   (m in log2 units)
-// The segments of b are the CTAs whose unit ranges meet b's units; slot = CTA + b.
-// grid (H, B, d/128), MERGE_THREADS threads: the split weights are computed once per
-// block into shared memory, then the warps split the partials among themselves (each
-// lane owning 4 consecutive dimensions) and are summed through shared memory.
-constexpr int MERGE_THREADS = 256;
-constexpr int MERGE_WARPS = MERGE_THREADS / 32;
-
-__global__ void __launch_bounds__(MERGE_THREADS) attn_merge_kernel(const Args a, int G,
-                                                                   uint16_t* out) {
-  extern __shared__ float s_w[];          // [G] split weights
-  __shared__ long long s_part[MERGE_WARPS][2];
-  __shared__ float s_red[MERGE_WARPS];
-  __shared__ float4 s_acc[MERGE_WARPS][32];
-  const int h = blockIdx.x, b = blockIdx.y, dchunk = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // prefix of units before b, and the batch total
-  long long before = 0, total = 0;
-  for (int i = tid; i < a.B; i += MERGE_THREADS) {
-    const int u = seq_units(a, i);
-    total += u;
-    if (i < b) before += u;
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    total += __shfl_xor_sync(0xffffffffu, total, o);
-    before += __shfl_xor_sync(0xffffffffu, before, o);
-  }
-  if (lane == 0) {
-    s_part[warp][0] = total;
-    s_part[warp][1] = before;
-  }
-  __syncthreads();
-  long long U = 0, P = 0;
-#pragma unroll
-  for (int w = 0; w < MERGE_WARPS; ++w) {
-    U += s_part[w][0];
-    P += s_part[w][1];
-  }
-  if (tid == 0 && h == 0 && dchunk == 0 && seq_malformed(a, b)) set_err(a.err, LSA_DEVERR_BAD_SIZE);
-  const int ub = seq_units(a, b);
-  const int d0 = dchunk * 128 + lane * 4;
-  uint16_t* dst = out + (static_cast<long long>(b) * a.H + h) * a.d + d0;
-  if (ub == 0) {
-    if (warp == 0) *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
-    return;
-  }
-  // CTA holding unit u: the largest c with floor(c*U/G) <= u; CTAs whose unit range is
-  // empty (grid larger than the work) hold no slot
-  const long long c_lo = ((P + 1) * G - 1) / U;
-  const long long c_hi = ((P + ub) * G - 1) / U;
-  const int n = static_cast<int>(c_hi - c_lo + 1);
-  float mx = -INFINITY;
-  for (int k = tid; k < n; k += MERGE_THREADS) {
-    const long long c = c_lo + k;
-    float m = -INFINITY;
-    if ((c * U) / G != ((c + 1) * U) / G) m = a.part_ml[((c + b) * a.H + h) * 2];
-    s_w[k] = m;
-    mx = fmaxf(mx, m);
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) s_red[warp] = mx;
-  __syncthreads();
-  float M = s_red[0];
-#pragma unroll
-  for (int w = 1; w < MERGE_WARPS; ++w) M = fmaxf(M, s_red[w]);
-  __syncthreads();
-  float ls = 0.f;
-  for (int k = tid; k < n; k += MERGE_THREADS) {
-    const long long c = c_lo + k;
-    const float m = s_w[k];
-    const float w = m == -INFINITY ? 0.f : exp2f(m - M);
-    if (w != 0.f) ls += w * a.part_ml[((c + b) * a.H + h) * 2 + 1];
-    s_w[k] = w;
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-  if (lane == 0) s_red[warp] = ls;
-  __syncthreads();
-  float lsum = 0.f;
-#pragma unroll
-  for (int w = 0; w < MERGE_WARPS; ++w) lsum += s_red[w];
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int k = warp; k < n; k += MERGE_WARPS) {
-    const float w = s_w[k];
-    if (w == 0.f) continue;
-    const long long slot = c_lo + k + b;
-    const float4 o = __ldcg(reinterpret_cast<const float4*>(a.part_o + (slot * a.H + h) * a.d + d0));
-    acc.x += w * o.x;
-    acc.y += w * o.y;
-    acc.z += w * o.z;
-    acc.w += w * o.w;
-  }
-  s_acc[warp][lane] = acc;
-  __syncthreads();
-  if (warp == 0) {
-    float4 t = s_acc[0][lane];
-#pragma unroll
-    for (int w = 1; w < MERGE_WARPS; ++w) {
-      const float4 v = s_acc[w][lane];
-      t.x += v.x;
-      t.y += v.y;
-      t.z += v.z;
-      t.w += v.w;
-    }
-    const float inv = 1.f / lsum;
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(t.x * inv, t.y * inv);
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(t.z * inv, t.w * inv);
-    uint2 pk;
-    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(dst) = pk;
+  // ring, Q and P buffers are free now: the merge reuses them
+  {
+    __shared__ long long s_U;
+    if (tid == 0) s_U = U;
+    __syncthreads();
+    uint32_t merge_bit = 0;
+    merge_phase(a, m, smem, LY::MISC_OFF, s_U, *abort != 0, merge_bit);
   }
 }
 
@@ -697,9 +854,12 @@ namespace {
 
 using lsa::attn::Args;
 
+// Workspace: fp32 partial O [G+B][H][d], partial (m, l) [G+B][H][2], then the two
+// grid-barrier counters on their own 256-byte line.
 size_t attn_ws_bytes(int B, int H, int d, int n_sm) {
   const size_t slots = static_cast<size_t>(n_sm) + static_cast<size_t>(B);
-  return slots * static_cast<size_t>(H) * (static_cast<size_t>(d) + 2) * sizeof(float);
+  const size_t body = slots * static_cast<size_t>(H) * (static_cast<size_t>(d) + 2) * sizeof(float);
+  return (body + 255) / 256 * 256 + 256;
 }
 
 template <int HP, int NDC>
@@ -716,8 +876,23 @@ lsa_status launch_attn(const CUtensorMap& mkv, const CUtensorMap& mq, const Args
       return LSA_ERR_CUDA;
     configured_device = dev;
   }
-  kern<<<G, lsa::attn::NTHREADS, LY::SMEM, stream>>>(mkv, mq, a);
-  return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+  // Cooperative launch: all G CTAs (one per SM) are resident together, which the
+  // fused merge's grid barrier relies on.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(lsa::attn::NTHREADS);
+  cfg.dynamicSmemBytes = LY::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mkv, mq, a) != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
+  return LSA_OK;
 }
 
 template <int HP>
@@ -734,6 +909,79 @@ lsa_status dispatch_d(const CUtensorMap& mkv, const CUtensorMap& mq, const Args&
 
 }  // namespace
 
+namespace lsa_host {
+
+lsa_status decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pages,
+                       const int32_t* block_table, int32_t bt_stride, const int32_t* n_entries,
+                       const int32_t* tail_len, int32_t B, int32_t H, int32_t d, float scale,
+                       uint16_t* out, void* ws, size_t ws_bytes, int32_t* err, void* stream,
+                       const AppendArgs* append) {
+  if (!q || !hbm_pool || !block_table || !n_entries || !out || !ws || !err)
+    return LSA_ERR_INVALID_ARG;
+  if (!append && !tail_len) return LSA_ERR_INVALID_ARG;
+  if (append && (!append->k_new || !append->v_new || append->tail < 1 || append->tail > 64))
+    return LSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || H > 64 || bt_stride <= 0 || n_pages <= 0) return LSA_ERR_INVALID_ARG;
+  if (d != 128 && d != 256 && d != 384 && d != 512) return LSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return LSA_ERR_INVALID_ARG;
+  if (n_pages > (int64_t(1) << 23)) return LSA_ERR_INVALID_ARG;  // page rows must fit in int32
+  if (static_cast<int64_t>(B) * H > (int64_t(1) << 30)) return LSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(hbm_pool) |
+       reinterpret_cast<uintptr_t>(ws)) & 15u)
+    return LSA_ERR_INVALID_ARG;
+  if (append && ((reinterpret_cast<uintptr_t>(append->k_new) |
+                  reinterpret_cast<uintptr_t>(append->v_new)) & 15u))
+    return LSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(out) & 1u) != 0) return LSA_ERR_INVALID_ARG;
+  const int G = sm_count();
+  if (G <= 0) return LSA_ERR_CUDA;
+  if (G > lsa::attn::MAX_GRID) return LSA_ERR_UNIMPLEMENTED;
+  if (ws_bytes < attn_ws_bytes(B, H, d, G)) return LSA_ERR_INVALID_ARG;
+  const int HP = (H + 15) / 16 * 16;
+  const int HPk = HP <= 16 ? 16 : HP <= 32 ? 32 : 64;
+
+  CUtensorMap mkv, mq;
+  lsa_status st = encode_tiled_2d(&mkv, hbm_pool, d, static_cast<uint64_t>(n_pages) * 128,
+                                  static_cast<uint64_t>(d) * 2, 64, lsa::attn::UNIT,
+                                  CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != LSA_OK) return st;
+  st = encode_tiled_2d(&mq, q, d, static_cast<uint64_t>(B) * H, static_cast<uint64_t>(d) * 2, 64,
+                       H, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != LSA_OK) return st;
+
+  Args a = {};
+  a.block_table = block_table;
+  a.n_entries = n_entries;
+  a.tail_len = tail_len;
+  a.part_o = static_cast<float*>(ws);
+  a.part_ml = a.part_o + (static_cast<size_t>(G) + B) * H * d;
+  const size_t body = (static_cast<size_t>(G) + B) * H * (static_cast<size_t>(d) + 2) * sizeof(float);
+  a.sync = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + (body + 255) / 256 * 256);
+  a.out = out;
+  a.pool = const_cast<uint16_t*>(hbm_pool);
+  if (append) {
+    a.k_new = append->k_new;
+    a.v_new = append->v_new;
+    a.tail_len_out = append->tail_len_out;
+    a.fused_tail = append->tail;
+  }
+  a.err = err;
+  a.n_pages = n_pages;
+  a.bt_stride = bt_stride;
+  a.B = B;
+  a.H = H;
+  a.d = d;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (HPk) {
+    case 16: return dispatch_d<16>(mkv, mq, a, G, s);
+    case 32: return dispatch_d<32>(mkv, mq, a, G, s);
+    default: return dispatch_d<64>(mkv, mq, a, G, s);
+  }
+}
+
+}  // namespace lsa_host
+
 extern "C" size_t lsa_decode_attn_workspace_size(int32_t B, int32_t H, int32_t d, int32_t n_sm) {
   if (B <= 0 || H <= 0 || d <= 0 || n_sm <= 0) return 0;
   return attn_ws_bytes(B, H, d, n_sm);
@@ -744,54 +992,6 @@ extern "C" lsa_status lsa_decode_attn(const uint16_t* q, const uint16_t* hbm_poo
                                       const int32_t* n_entries, const int32_t* tail_len,
                                       int32_t B, int32_t H, int32_t d, float scale, uint16_t* out,
                                       void* ws, size_t ws_bytes, int32_t* err, void* stream) {
-  if (!q || !hbm_pool || !block_table || !n_entries || !tail_len || !out || !ws || !err)
-    return LSA_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || H > 64 || bt_stride <= 0 || n_pages <= 0) return LSA_ERR_INVALID_ARG;
-  if (d != 128 && d != 256 && d != 384 && d != 512) return LSA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !isfinite(scale)) return LSA_ERR_INVALID_ARG;
-  if (n_pages > (int64_t(1) << 23)) return LSA_ERR_INVALID_ARG;  // page rows must fit in int32
-  if (static_cast<int64_t>(B) * H > (int64_t(1) << 30)) return LSA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(hbm_pool) |
-       reinterpret_cast<uintptr_t>(ws)) & 15u)
-    return LSA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(out) & 7u) != 0) return LSA_ERR_INVALID_ARG;
-  const int G = lsa_host::sm_count();
-  if (G <= 0) return LSA_ERR_CUDA;
-  if (ws_bytes < attn_ws_bytes(B, H, d, G)) return LSA_ERR_INVALID_ARG;
-  const int HP = (H + 15) / 16 * 16;
-  const int HPk = HP <= 16 ? 16 : HP <= 32 ? 32 : 64;
-
-  CUtensorMap mkv, mq;
-  lsa_status st = lsa_host::encode_tiled_2d(&mkv, hbm_pool, d, static_cast<uint64_t>(n_pages) * 128,
-                                            static_cast<uint64_t>(d) * 2, 64, lsa::attn::UNIT,
-                                            CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != LSA_OK) return st;
-  st = lsa_host::encode_tiled_2d(&mq, q, d, static_cast<uint64_t>(B) * H,
-                                 static_cast<uint64_t>(d) * 2, 64, H,
-                                 CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != LSA_OK) return st;
-
-  Args a;
-  a.block_table = block_table;
-  a.n_entries = n_entries;
-  a.tail_len = tail_len;
-  a.part_o = static_cast<float*>(ws);
-  a.part_ml = a.part_o + (static_cast<size_t>(G) + B) * H * d;
-  a.err = err;
-  a.n_pages = n_pages;
-  a.bt_stride = bt_stride;
-  a.B = B;
-  a.H = H;
-  a.d = d;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  switch (HPk) {
-    case 16: st = dispatch_d<16>(mkv, mq, a, G, s); break;
-    case 32: st = dispatch_d<32>(mkv, mq, a, G, s); break;
-    default: st = dispatch_d<64>(mkv, mq, a, G, s); break;
-  }
-  if (st != LSA_OK) return st;
-  lsa::attn::attn_merge_kernel<<<dim3(H, B, d / 128), lsa::attn::MERGE_THREADS,
-                                 G * sizeof(float), s>>>(a, G, out);
-  return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+  return lsa_host::decode_attn(q, hbm_pool, n_pages, block_table, bt_stride, n_entries, tail_len,
+                               B, H, d, scale, out, ws, ws_bytes, err, stream, nullptr);
 }

@@ -135,6 +135,28 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Order this thread's generic-proxy global-memory writes before later async-proxy
+// (TMA) reads of the same addresses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16), completing
+// on an mbarrier's transaction count.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Order this thread's generic-proxy shared-memory writes before later async-proxy
 // (tensor core / TMA) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -263,5 +285,24 @@ int sm_count();
 lsa_status encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                            CUtensorMapSwizzle swizzle);
+
+// Fused token append for the decode-step path: k_new / v_new [B][d] go into slot
+// tail-1 of each sequence's last block-table page; tail_len_out receives `tail`.
+struct AppendArgs {
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  int32_t* tail_len_out;
+  int tail;
+};
+
+// lsa_decode_attn with an optional fused append (defined in lsa_attn.cu).
+lsa_status decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pages,
+                       const int32_t* block_table, int32_t bt_stride, const int32_t* n_entries,
+                       const int32_t* tail_len, int32_t B, int32_t H, int32_t d, float scale,
+                       uint16_t* out, void* ws, size_t ws_bytes, int32_t* err, void* stream,
+                       const AppendArgs* append);
+
+// Device-visible address of pinned host memory, or nullptr (defined in lsa_gather.cu).
+const void* mapped_host_ptr(const void* p);
 
 }  // namespace lsa_host

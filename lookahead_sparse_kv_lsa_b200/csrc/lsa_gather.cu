@@ -161,6 +161,18 @@ __global__ void __launch_bounds__(THREADS) pass_setup_kernel(const StepArgs a, i
   for (long long i = tid; i < nb - first + 1; i += THREADS)
     a.res_pages[static_cast<long long>(b) * (a.wb + 1) + i] =
         static_cast<int32_t>(ring_page(a, b, first + i));
+  // the previous pass's tail page is complete: write it back to the cold pool
+  if (p > 0) {
+    const long long hb = __ldg(a.host_blk_off + b) + nb - 1;
+    if (hb < __ldg(a.host_blk_off + b + 1) && hb < a.host_blocks) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.hbm_pool + ring_page(a, b, nb - 1) * 128 * a.d);
+      uint4* dst = reinterpret_cast<uint4*>(a.host_pool + hb * 128 * a.d);
+      for (int i = tid; i < 16 * a.d; i += THREADS) dst[i] = src[i];
+    } else if (tid == 0) {
+      set_err(a.err, LSA_DEVERR_BAD_PAGE);
+    }
+    __syncthreads();  // with a one-page ring the new tail page is the old one
+  }
   uint4* tail = reinterpret_cast<uint4*>(a.hbm_pool + ring_page(a, b, nb) * 128 * a.d);
   for (int i = tid; i < 16 * a.d; i += THREADS) tail[i] = make_uint4(0u, 0u, 0u, 0u);
 }
@@ -329,6 +341,23 @@ extern "C" lsa_status lsa_append(const lsa_state* st, int64_t step, const uint16
   return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
 }
 
+extern "C" lsa_status lsa_decode_step(const lsa_state* st, int64_t step, const uint16_t* q,
+                                      const uint16_t* k_new, const uint16_t* v_new, uint16_t* out,
+                                      void* stream) {
+  const lsa_status v = lsa_state_check(st);
+  if (v != LSA_OK) return v;
+  if (step < 0 || step / LSA_TAU > (int64_t(1) << 30) || !q || !k_new || !v_new || !out)
+    return LSA_ERR_INVALID_ARG;
+  lsa_host::AppendArgs ap;
+  ap.k_new = k_new;
+  ap.v_new = v_new;
+  ap.tail_len_out = st->tail_len;
+  ap.tail = static_cast<int>(step % LSA_TAU) + 1;
+  return lsa_host::decode_attn(q, st->hbm_pool, st->n_pages, st->block_table, st->bt_stride,
+                               st->n_entries, st->tail_len, st->B, st->H, st->d, st->scale, out,
+                               st->attn_ws, st->attn_ws_bytes, st->err, stream, &ap);
+}
+
 extern "C" lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t* h,
                                const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
                                uint16_t* out, void* stream) {
@@ -354,9 +383,5 @@ extern "C" lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t
                    st->n_entries, st->err, stream);
     if (v != LSA_OK) return v;
   }
-  v = lsa_append(st, step, k_new, v_new, stream);
-  if (v != LSA_OK) return v;
-  return lsa_decode_attn(q, st->hbm_pool, st->n_pages, st->block_table, st->bt_stride,
-                         st->n_entries, st->tail_len, st->B, st->H, st->d, st->scale, out,
-                         st->attn_ws, st->attn_ws_bytes, st->err, stream);
+  return lsa_decode_step(st, step, q, k_new, v_new, out, stream);
 }

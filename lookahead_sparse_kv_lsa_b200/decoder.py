@@ -111,6 +111,10 @@ class LsaDecoder:
         from . import lsa_append
         lsa_append(self.state, step, k_new, v_new, stream)
 
+    def decode_step(self, step: int, q, k_new, v_new, out, stream=None) -> None:
+        from . import lsa_decode_step
+        lsa_decode_step(self.state, step, q, k_new, v_new, out, stream)
+
     def attend(self, q, out, stream=None) -> None:
         from . import lsa_decode_attn
         lsa_decode_attn(q, self.hbm_pool, self.block_table, self.n_entries, self.tail_len,
