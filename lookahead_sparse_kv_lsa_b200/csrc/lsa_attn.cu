@@ -58,6 +58,7 @@ struct Misc {
   float alpha[64];
   // fused merge
   int n_items, total_items;
+  long long merge_j0, merge_j1;
   int item_b[MAXITEMS], item_h[MAXITEMS], item_clo[MAXITEMS], item_chi[MAXITEMS];
   float wgt[MAX_GRID];
 };
@@ -206,17 +207,50 @@ __device__ __forceinline__ bool cta_empty(long long c, long long U, long long G)
   return (c * U) / G == ((c + 1) * U) / G;
 }
 
-// Warp 0: list this CTA's merge items for round `round`. Items are the (sequence, head)
-// pairs of every sequence whose units span more than one CTA, numbered in sequence
-// order; item j belongs to CTA j % G. Returns the batch's item total (all lanes).
-__device__ __noinline__ int plan_merge(const Args& a, long long U, int round, Misc* m, int lane) {
+// Merge work items are (sequence, head, 64-dim chunk) triples of every sequence whose
+// units span more than one CTA (they are merged from partials) or that has no units at
+// all (its output is zero-filled), numbered in sequence order. CTA c owns the
+// contiguous item range [c*T/G, (c+1)*T/G), so a CTA's items mostly share a head.
+//
+// Warp 0: record the sequences that meet this CTA's item range, skipping the first
+// `skip` of them (at most MAXITEMS are recorded). Also reports malformed sequences
+// (each from one CTA only).
+__device__ __noinline__ void plan_merge(const Args& a, long long U, int skip, Misc* m, int lane) {
   const long long G = gridDim.x;
   const int cta = blockIdx.x;
-  long long base_u = 0;
-  int base_item = 0, mine = 0;
-  for (int b0 = 0; b0 < a.B; b0 += 32) {
+  const int n_chunks = a.d / 64;
+  // pass 1: total items T
+  long long T = 0;
+  {
+    long long base_u = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+      const int b = b0 + lane;
+      const int u = b < a.B ? seq_units(a, b) : 0;
+      long long incl = u;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const long long p = base_u + incl - u;
+      bool has = false;
+      if (b < a.B) has = (u == 0) || (cta_of_unit(p, U, G) != cta_of_unit(p + u - 1, U, G));
+      long long items = has ? static_cast<long long>(a.H) * n_chunks : 0;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) items += __shfl_xor_sync(0xffffffffu, items, o);
+      T += items;
+      base_u += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  const long long j0 = (static_cast<long long>(cta) * T) / G;
+  const long long j1 = (static_cast<long long>(cta + 1) * T) / G;
+  // pass 2: sequences meeting [j0, j1)
+  long long base_u = 0, base_i = 0;
+  int found = 0;
+  for (int b0 = 0; b0 < a.B && base_i < j1; b0 += 32) {
     const int b = b0 + lane;
     const int u = b < a.B ? seq_units(a, b) : 0;
+    if (b < a.B && b % G == cta && seq_malformed(a, b)) set_err(a.err, LSA_DEVERR_BAD_SIZE);
     long long incl = u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -224,46 +258,47 @@ __device__ __noinline__ int plan_merge(const Args& a, long long U, int round, Mi
       if (lane >= o) incl += t;
     }
     const long long p = base_u + incl - u;
-    long long clo = 0, chi = 0;
-    bool split = false;
-    if (u > 0) {
-      clo = cta_of_unit(p, U, G);
-      chi = cta_of_unit(p + u - 1, U, G);
-      split = clo != chi;
-    }
-    const int items = split ? a.H : 0;
-    int iincl = items;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, iincl, o);
-      if (lane >= o) iincl += t;
-    }
-    const int ibase = base_item + iincl - items;
-    if (items > 0) {
-      // first item of this sequence owned by this CTA, then every G-th
-      int j = ibase + static_cast<int>(((cta - ibase) % G + G) % G);
-      for (; j < ibase + items; j += static_cast<int>(G)) {
-        const int rank = (j - cta) / static_cast<int>(G) - round * MAXITEMS;
-        if (rank >= 0 && rank < MAXITEMS) {
-          m->item_b[rank] = b;
-          m->item_h[rank] = j - ibase;
-          m->item_clo[rank] = static_cast<int>(clo);
-          m->item_chi[rank] = static_cast<int>(chi);
-        }
+    long long clo = 0, chi = -1;
+    bool has = false;
+    if (b < a.B) {
+      if (u == 0) {
+        has = true;
+      } else {
+        clo = cta_of_unit(p, U, G);
+        chi = cta_of_unit(p + u - 1, U, G);
+        has = clo != chi;
       }
     }
+    const long long items = has ? static_cast<long long>(a.H) * n_chunks : 0;
+    long long iincl = items;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long t = __shfl_up_sync(0xffffffffu, iincl, o);
+      if (lane >= o) iincl += t;
+    }
+    const long long ib = base_i + iincl - items;
+    const bool hit = items > 0 && ib < j1 && ib + items > j0;
+    const unsigned mask = __ballot_sync(0xffffffffu, hit);
+    if (hit) {
+      const int idx = found + __popc(mask & ((1u << lane) - 1u)) - skip;
+      if (idx >= 0 && idx < MAXITEMS) {
+        m->item_b[idx] = b;
+        m->item_h[idx] = static_cast<int>(ib);  // first item of the sequence
+        m->item_clo[idx] = static_cast<int>(clo);
+        m->item_chi[idx] = static_cast<int>(chi);
+      }
+    }
+    found += __popc(mask);
     base_u += __shfl_sync(0xffffffffu, incl, 31);
-    base_item += __shfl_sync(0xffffffffu, iincl, 31);
+    base_i += __shfl_sync(0xffffffffu, iincl, 31);
   }
-  // items of this CTA: those j < base_item with j % G == cta
-  const int total = base_item;
-  if (total > cta) mine = (total - cta + static_cast<int>(G) - 1) / static_cast<int>(G);
   if (lane == 0) {
-    m->total_items = total;
-    const int left = mine - round * MAXITEMS;
+    const int left = found - skip;
     m->n_items = left < 0 ? 0 : (left > MAXITEMS ? MAXITEMS : left);
+    m->total_items = static_cast<int>(T > 0x7fffffff ? 0x7fffffff : T);
+    m->merge_j0 = j0;
+    m->merge_j1 = j1;
   }
-  return total;
 }
 
 // Block-wide reductions over the CTA's threads through m->red[0][*].
@@ -291,19 +326,21 @@ __device__ __forceinline__ float block_sum(float v, Misc* m, int tid, int nwarps
 // Fused log-sum-exp merge, run by every thread of every CTA after its segments:
 //   M = max_k m_k,  out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k   (m in log2 units)
 // over the partials k of a split sequence. A grid-wide barrier (one arrival counter,
-// bounded wait) separates the partial writes from the reads; the partial rows of one
-// (sequence, head) item are brought into shared memory with 1-D bulk copies, then
-// every thread reduces a slice of the head dimension over all partials.
-__device__ __noinline__ void merge_phase(const Args& a, Misc* m, uint8_t* buf, int buf_bytes, long long U,
-                            bool aborted, uint32_t& merge_phase_bit) {
+// bounded wait) separates the partial writes from the reads. For each item the 16
+// float4 columns of a 64-dim chunk are spread over the threads together with the
+// partials (MERGE_RG row groups), loads issued back to back, and the row groups summed
+// through shared memory.
+constexpr int MERGE_RG = NTHREADS / 16;
+
+__device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* scratch, long long U,
+                                         bool aborted) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nthr = blockDim.x, nwarps = nthr >> 5;
+  const int nwarps = NTHREADS / 32;
   const long long G = gridDim.x;
-  volatile int* abort = &m->abort;
+  const int n_chunks = a.d / 64;
   if (warp == 0) plan_merge(a, U, 0, m, lane);
   __syncthreads();
-  const int total = m->total_items;
-  if (total == 0) return;             // nothing split: no barrier, every CTA agrees
+  if (m->total_items == 0) return;     // nothing split or empty: no barrier, all CTAs agree
   // ---- grid barrier: all partials written before any is read
   if (tid == 0) {
     __threadfence();
@@ -311,91 +348,104 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, uint8_t* buf, i
     const uint64_t t0 = globaltimer_ns();
     bool ok = true;
     while (ld_acquire_gpu(a.sync) < static_cast<unsigned int>(G)) {
+      __nanosleep(64);
       if (globaltimer_ns() - t0 > LSA_WAIT_LIMIT_NS) {
         ok = false;
         break;
       }
     }
     __threadfence();
-    fence_proxy_async_global();       // the partials are read back by bulk copies
     if (!ok) {
       set_err(a.err, LSA_DEVERR_TIMEOUT);
-      *abort = 1;
+      m->abort = 1;
     }
   }
   __syncthreads();
-  bool failed = *abort != 0 || aborted;   // the same value in every thread
+  const bool failed = m->abort != 0 || aborted;   // the same value in every thread
   if (!failed) {
-    float* fbuf = reinterpret_cast<float*>(buf);
+    const long long j0 = m->merge_j0, j1 = m->merge_j1;
+    const int col = tid & 15, rg = tid >> 4;         // float4 column, row group
+    int cached_b = -1, cached_h = -1;
+    float inv_l = 0.f;
     for (int round = 0;; ++round) {
       if (round > 0) {
         __syncthreads();
-        if (warp == 0) plan_merge(a, U, round, m, lane);
+        if (warp == 0) plan_merge(a, U, round * MAXITEMS, m, lane);
         __syncthreads();
       }
-      const int n_items = m->n_items;
-      if (n_items == 0) break;
-      for (int it = 0; it < n_items && !failed; ++it) {
-        const int b = m->item_b[it], h = m->item_h[it];
-        const int clo = m->item_clo[it], n = m->item_chi[it] - clo + 1;
-        // split weights
-        float mx = -INFINITY;
-        for (int k = tid; k < n; k += nthr) {
-          const long long c = clo + k;
-          const float mk =
-              cta_empty(c, U, G) ? -INFINITY : __ldcg(a.part_ml + ((c + b) * a.H + h) * 2);
-          m->wgt[k] = mk;
-          mx = fmaxf(mx, mk);
-        }
-        const float M = block_max(mx, m, tid, nwarps);
-        float ls = 0.f;
-        for (int k = tid; k < n; k += nthr) {
-          const long long c = clo + k;
-          const float mk = m->wgt[k];
-          const float w = mk == -INFINITY ? 0.f : exp2f(mk - M);
-          if (w != 0.f) ls += w * __ldcg(a.part_ml + ((c + b) * a.H + h) * 2 + 1);
-          m->wgt[k] = w;
-        }
-        const float inv_l = 1.f / block_sum(ls, m, tid, nwarps);
-        // partial rows, in chunks of the head dimension that fit the buffer
-        int chunk = (buf_bytes / (n * 4)) / 32 * 32;
-        if (chunk > a.d) chunk = a.d;
-        for (int d0 = 0; d0 < a.d && !failed; d0 += chunk) {
-          const int cw = min(chunk, a.d - d0);
-          if (tid == 0) {
-            fence_proxy_async_smem();     // earlier generic accesses of the buffer first
-            uint32_t bytes = 0;
-            for (int k = 0; k < n; ++k)
-              if (m->wgt[k] != 0.f) bytes += cw * 4;
-            mbar_arrive_expect_tx(&m->merge_bar, bytes);
-            for (int k = 0; k < n; ++k) {
-              if (m->wgt[k] == 0.f) continue;
-              const long long slot = clo + k + b;
-              bulk_load(fbuf + static_cast<long long>(k) * cw,
-                        a.part_o + (slot * a.H + h) * a.d + d0, cw * 4, &m->merge_bar);
-            }
+      const int nrec = m->n_items;
+      if (nrec == 0) break;
+      for (int r = 0; r < nrec; ++r) {
+        const int b = m->item_b[r];
+        const long long ib = m->item_h[r];
+        const int clo = m->item_clo[r], n = m->item_chi[r] - clo + 1;
+        const long long lo = j0 > ib ? j0 : ib;
+        const long long hi = j1 < ib + static_cast<long long>(a.H) * n_chunks
+                                 ? j1 : ib + static_cast<long long>(a.H) * n_chunks;
+        for (long long j = lo; j < hi; ++j) {
+          const int h = static_cast<int>((j - ib) / n_chunks);
+          const int chunk = static_cast<int>((j - ib) % n_chunks);
+          uint16_t* dst = a.out + (static_cast<long long>(b) * a.H + h) * a.d + chunk * 64;
+          if (n <= 0) {                  // a sequence with no tokens: zeros
+            if (tid < 32) reinterpret_cast<uint32_t*>(dst)[tid] = 0u;
+            continue;
           }
-          const bool ok = __syncthreads_and(mbar_wait(&m->merge_bar, merge_phase_bit, nullptr)) != 0;
-          merge_phase_bit ^= 1u;
-          if (!ok) {
-            failed = true;
-            if (tid == 0) set_err(a.err, LSA_DEVERR_TIMEOUT);
-          } else {
-            uint16_t* dst = a.out + (static_cast<long long>(b) * a.H + h) * a.d + d0;
-            for (int j = tid; j < cw; j += nthr) {
-              float acc = 0.f;
-              for (int k = 0; k < n; ++k) {
-                const float w = m->wgt[k];
-                if (w != 0.f) acc += w * fbuf[static_cast<long long>(k) * cw + j];
-              }
-              const __nv_bfloat16 v = __float2bfloat16_rn(acc * inv_l);
-              dst[j] = *reinterpret_cast<const uint16_t*>(&v);
+          if (b != cached_b || h != cached_h) {   // split weights of this head
+            float mx = -INFINITY;
+            for (int k = tid; k < n; k += NTHREADS) {
+              const long long c = clo + k;
+              const float mk =
+                  cta_empty(c, U, G) ? -INFINITY : __ldcg(a.part_ml + ((c + b) * a.H + h) * 2);
+              m->wgt[k] = mk;
+              mx = fmaxf(mx, mk);
             }
+            const float M = block_max(mx, m, tid, nwarps);
+            float ls = 0.f;
+            for (int k = tid; k < n; k += NTHREADS) {
+              const long long c = clo + k;
+              const float mk = m->wgt[k];
+              const float w = mk == -INFINITY ? 0.f : exp2f(mk - M);
+              if (w != 0.f) ls += w * __ldcg(a.part_ml + ((c + b) * a.H + h) * 2 + 1);
+              m->wgt[k] = w;
+            }
+            inv_l = 1.f / block_sum(ls, m, tid, nwarps);  // ends with a barrier: wgt visible
+            cached_b = b;
+            cached_h = h;
           }
-          __syncthreads();  // the buffer is refilled by the next chunk
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          const float* col_base = a.part_o + (static_cast<long long>(h) * a.d + chunk * 64 + col * 4);
+#pragma unroll 8
+          for (int k = rg; k < n; k += MERGE_RG) {
+            const float w = m->wgt[k];
+            const long long slot = clo + k + b;
+            const float4 o = __ldcg(reinterpret_cast<const float4*>(col_base + slot * a.H * a.d));
+            acc.x += w * o.x;
+            acc.y += w * o.y;
+            acc.z += w * o.z;
+            acc.w += w * o.w;
+          }
+          reinterpret_cast<float4*>(scratch)[rg * 16 + col] = acc;
+          __syncthreads();
+          if (tid < 16) {
+            float4 t = reinterpret_cast<float4*>(scratch)[tid];
+            for (int g = 1; g < MERGE_RG; ++g) {
+              const float4 v = reinterpret_cast<float4*>(scratch)[g * 16 + tid];
+              t.x += v.x;
+              t.y += v.y;
+              t.z += v.z;
+              t.w += v.w;
+            }
+            const __nv_bfloat162 p0 = __floats2bfloat162_rn(t.x * inv_l, t.y * inv_l);
+            const __nv_bfloat162 p1 = __floats2bfloat162_rn(t.z * inv_l, t.w * inv_l);
+            uint2 pk;
+            pk.x = *reinterpret_cast<const uint32_t*>(&p0);
+            pk.y = *reinterpret_cast<const uint32_t*>(&p1);
+            reinterpret_cast<uint2*>(dst)[tid] = pk;
+          }
+          __syncthreads();
         }
       }
-      if (failed || m->n_items < MAXITEMS) break;
+      if (nrec < MAXITEMS) break;
     }
   }
   // ---- departure: the last CTA out resets the counters for the next launch
@@ -841,8 +891,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __shared__ long long s_U;
     if (tid == 0) s_U = U;
     __syncthreads();
-    uint32_t merge_bit = 0;
-    merge_phase(a, m, smem, LY::MISC_OFF, s_U, *abort != 0, merge_bit);
+    merge_phase(a, m, reinterpret_cast<float*>(smem), s_U, *abort != 0);
   }
 }
 
