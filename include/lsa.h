@@ -148,7 +148,9 @@ lsa_status lsa_gather(const uint16_t* host_pool, int64_t host_blocks,
  *   ws          device workspace of lsa_decode_attn_workspace_size(B, H, d, n_sm)
  *               bytes, n_sm = multiprocessor count of the current device
  * Supported: d in {128, 256, 384, 512}, 1 <= H <= 64, scale > 0, n_pages <= 2^23,
- *            q, hbm_pool and ws 16-byte aligned, out 8-byte aligned.
+ *            q, hbm_pool, ws and out 16-byte aligned. The launch is cooperative (one
+ *            CTA per SM, all resident): the partial results are merged inside the same
+ *            kernel behind a grid-wide barrier whose counters live in ws.
  */
 lsa_status lsa_decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pages,
                            const int32_t* block_table, int32_t bt_stride,

@@ -38,7 +38,8 @@ constexpr int STAGE_BYTES = TILE * 128;   // [128 rows][64 bf16] = 16 KB
 constexpr int NTHREADS = 192;
 constexpr int MAXSEG = 16;                // segments planned per batch
 constexpr float RESCALE_LOG2 = 8.0f;      // raise the running max only by more than 2^8
-constexpr int MAXITEMS = 32;              // merge items (sequence, head) per CTA and round
+constexpr int MAXITEMS = 64;              // sequences a CTA's merge range meets, per round
+constexpr int MAXRUNS = 32;               // (sequence, head, chunk range) runs per merge group
 constexpr int MAX_GRID = 256;             // CTAs per launch (one per SM)
 
 struct Seg {
@@ -58,9 +59,13 @@ struct Misc {
   float alpha[64];
   // fused merge
   int n_items, total_items;
-  long long merge_j0, merge_j1;
+  long long merge_j0, merge_j1, cur_j;
+  int cur_rec, n_runs, group_floats;
+  uint32_t group_bytes;
   int item_b[MAXITEMS], item_h[MAXITEMS], item_clo[MAXITEMS], item_chi[MAXITEMS];
-  float wgt[MAX_GRID];
+  int run_b[MAXRUNS], run_h[MAXRUNS], run_d0[MAXRUNS], run_w[MAXRUNS], run_clo[MAXRUNS],
+      run_n[MAXRUNS], run_off[MAXRUNS];
+  float run_inv[MAXRUNS];
 };
 
 struct Args {
@@ -326,18 +331,17 @@ __device__ __forceinline__ float block_sum(float v, Misc* m, int tid, int nwarps
 // Fused log-sum-exp merge, run by every thread of every CTA after its segments:
 //   M = max_k m_k,  out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k   (m in log2 units)
 // over the partials k of a split sequence. A grid-wide barrier (one arrival counter,
-// bounded wait) separates the partial writes from the reads. For each item the 16
-// float4 columns of a 64-dim chunk are spread over the threads together with the
-// partials (MERGE_RG row groups), loads issued back to back, and the row groups summed
-// through shared memory.
-constexpr int MERGE_RG = NTHREADS / 16;
-
-__device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* scratch, long long U,
-                                         bool aborted) {
+// bounded wait) separates the partial writes from the reads. The CTA's items are cut
+// into runs (one sequence, one head, a range of 64-dim chunks); a group of runs that
+// fits the idle shared memory has all its partial rows fetched with 1-D bulk copies
+// (issued by all threads, one round trip) while one warp per run derives the split
+// weights; then every thread reduces a few output dimensions over the partials.
+__device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int buf_floats,
+                                         long long U, bool aborted) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = NTHREADS / 32;
+  constexpr int NWARPS = NTHREADS / 32;
   const long long G = gridDim.x;
-  const int n_chunks = a.d / 64;
+  const int nch = a.d / 64;
   if (warp == 0) plan_merge(a, U, 0, m, lane);
   __syncthreads();
   if (m->total_items == 0) return;     // nothing split or empty: no barrier, all CTAs agree
@@ -348,105 +352,159 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* scratch,
     const uint64_t t0 = globaltimer_ns();
     bool ok = true;
     while (ld_acquire_gpu(a.sync) < static_cast<unsigned int>(G)) {
-      __nanosleep(64);
+      __nanosleep(32);
       if (globaltimer_ns() - t0 > LSA_WAIT_LIMIT_NS) {
         ok = false;
         break;
       }
     }
     __threadfence();
+    fence_proxy_async_global();       // the partials are read back by bulk copies
     if (!ok) {
       set_err(a.err, LSA_DEVERR_TIMEOUT);
       m->abort = 1;
     }
   }
   __syncthreads();
-  const bool failed = m->abort != 0 || aborted;   // the same value in every thread
-  if (!failed) {
-    const long long j0 = m->merge_j0, j1 = m->merge_j1;
-    const int col = tid & 15, rg = tid >> 4;         // float4 column, row group
-    int cached_b = -1, cached_h = -1;
-    float inv_l = 0.f;
-    for (int round = 0;; ++round) {
-      if (round > 0) {
-        __syncthreads();
-        if (warp == 0) plan_merge(a, U, round * MAXITEMS, m, lane);
-        __syncthreads();
-      }
-      const int nrec = m->n_items;
-      if (nrec == 0) break;
-      for (int r = 0; r < nrec; ++r) {
-        const int b = m->item_b[r];
-        const long long ib = m->item_h[r];
-        const int clo = m->item_clo[r], n = m->item_chi[r] - clo + 1;
-        const long long lo = j0 > ib ? j0 : ib;
-        const long long hi = j1 < ib + static_cast<long long>(a.H) * n_chunks
-                                 ? j1 : ib + static_cast<long long>(a.H) * n_chunks;
-        for (long long j = lo; j < hi; ++j) {
-          const int h = static_cast<int>((j - ib) / n_chunks);
-          const int chunk = static_cast<int>((j - ib) % n_chunks);
-          uint16_t* dst = a.out + (static_cast<long long>(b) * a.H + h) * a.d + chunk * 64;
-          if (n <= 0) {                  // a sequence with no tokens: zeros
-            if (tid < 32) reinterpret_cast<uint32_t*>(dst)[tid] = 0u;
+  bool failed = m->abort != 0 || aborted;   // the same value in every thread
+  uint32_t phase = 0;
+  for (int round = 0; !failed; ++round) {
+    if (round > 0) {
+      __syncthreads();
+      if (warp == 0) plan_merge(a, U, round * MAXITEMS, m, lane);
+      __syncthreads();
+    }
+    const int nrec = m->n_items;
+    if (nrec == 0) break;
+    if (tid == 0) {
+      m->cur_rec = 0;
+      m->cur_j = -1;
+    }
+    __syncthreads();
+    while (!failed) {
+      // ---- thread 0 cuts the next group of runs
+      if (tid == 0) {
+        int r = m->cur_rec, nr = 0;
+        long long j = m->cur_j;
+        long long used = 0;
+        while (r < nrec && nr < MAXRUNS) {
+          const long long ib = m->item_h[r];
+          const long long lo = m->merge_j0 > ib ? m->merge_j0 : ib;
+          const long long hi_all = ib + static_cast<long long>(a.H) * nch;
+          const long long hi = m->merge_j1 < hi_all ? m->merge_j1 : hi_all;
+          if (j < lo) j = lo;
+          if (j >= hi) {
+            ++r;
+            j = -1;
             continue;
           }
-          if (b != cached_b || h != cached_h) {   // split weights of this head
-            float mx = -INFINITY;
-            for (int k = tid; k < n; k += NTHREADS) {
-              const long long c = clo + k;
-              const float mk =
-                  cta_empty(c, U, G) ? -INFINITY : __ldcg(a.part_ml + ((c + b) * a.H + h) * 2);
-              m->wgt[k] = mk;
-              mx = fmaxf(mx, mk);
-            }
-            const float M = block_max(mx, m, tid, nwarps);
-            float ls = 0.f;
-            for (int k = tid; k < n; k += NTHREADS) {
-              const long long c = clo + k;
-              const float mk = m->wgt[k];
-              const float w = mk == -INFINITY ? 0.f : exp2f(mk - M);
-              if (w != 0.f) ls += w * __ldcg(a.part_ml + ((c + b) * a.H + h) * 2 + 1);
-              m->wgt[k] = w;
-            }
-            inv_l = 1.f / block_sum(ls, m, tid, nwarps);  // ends with a barrier: wgt visible
-            cached_b = b;
-            cached_h = h;
+          const int h = static_cast<int>((j - ib) / nch);
+          const int c0 = static_cast<int>((j - ib) % nch);
+          long long run_end = ib + static_cast<long long>(h + 1) * nch;
+          if (run_end > hi) run_end = hi;
+          int nchunks = static_cast<int>(run_end - j);
+          const int n = m->item_chi[r] - m->item_clo[r] + 1;   // 0: empty sequence
+          long long need = static_cast<long long>(n) * (nchunks * 64) + n;
+          if (used + need > buf_floats) {
+            if (nr > 0) break;
+            nchunks = static_cast<int>((buf_floats / (n > 0 ? n : 1) - 1) / 64);
+            if (nchunks < 1) nchunks = 1;  // buf_floats >= 256 * 65 by construction
+            need = static_cast<long long>(n) * (nchunks * 64) + n;
           }
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          const float* col_base = a.part_o + (static_cast<long long>(h) * a.d + chunk * 64 + col * 4);
-#pragma unroll 8
-          for (int k = rg; k < n; k += MERGE_RG) {
-            const float w = m->wgt[k];
-            const long long slot = clo + k + b;
-            const float4 o = __ldcg(reinterpret_cast<const float4*>(col_base + slot * a.H * a.d));
-            acc.x += w * o.x;
-            acc.y += w * o.y;
-            acc.z += w * o.z;
-            acc.w += w * o.w;
-          }
-          reinterpret_cast<float4*>(scratch)[rg * 16 + col] = acc;
-          __syncthreads();
-          if (tid < 16) {
-            float4 t = reinterpret_cast<float4*>(scratch)[tid];
-            for (int g = 1; g < MERGE_RG; ++g) {
-              const float4 v = reinterpret_cast<float4*>(scratch)[g * 16 + tid];
-              t.x += v.x;
-              t.y += v.y;
-              t.z += v.z;
-              t.w += v.w;
-            }
-            const __nv_bfloat162 p0 = __floats2bfloat162_rn(t.x * inv_l, t.y * inv_l);
-            const __nv_bfloat162 p1 = __floats2bfloat162_rn(t.z * inv_l, t.w * inv_l);
-            uint2 pk;
-            pk.x = *reinterpret_cast<const uint32_t*>(&p0);
-            pk.y = *reinterpret_cast<const uint32_t*>(&p1);
-            reinterpret_cast<uint2*>(dst)[tid] = pk;
-          }
-          __syncthreads();
+          m->run_b[nr] = m->item_b[r];
+          m->run_h[nr] = h;
+          m->run_d0[nr] = c0 * 64;
+          m->run_w[nr] = nchunks * 64;
+          m->run_clo[nr] = m->item_clo[r];
+          m->run_n[nr] = n;
+          m->run_off[nr] = static_cast<int>(used);
+          used += need;
+          j += nchunks;
+          ++nr;
+        }
+        m->cur_rec = r;
+        m->cur_j = j;
+        m->n_runs = nr;
+        m->group_floats = static_cast<int>(used);
+        uint32_t bytes = 0;
+        for (int q = 0; q < nr; ++q) bytes += static_cast<uint32_t>(m->run_n[q]) * m->run_w[q] * 4u;
+        m->group_bytes = bytes;
+        if (bytes > 0) {
+          fence_proxy_async_smem();     // earlier generic accesses of the buffer first
+          mbar_arrive_expect_tx(&m->merge_bar, bytes);
         }
       }
-      if (nrec < MAXITEMS) break;
+      __syncthreads();
+      const int nr = m->n_runs;
+      if (nr == 0) break;
+      // ---- partial rows: one bulk copy per (run, split), spread over all threads
+      int total_rows = 0;
+      for (int q = 0; q < nr; ++q) total_rows += m->run_n[q];
+      fence_proxy_async_smem();         // this thread's earlier reads of the buffer first
+      for (int t = tid; t < total_rows; t += NTHREADS) {
+        int q = 0, k = t;
+        while (k >= m->run_n[q]) k -= m->run_n[q++];
+        const long long slot = m->run_clo[q] + k + m->run_b[q];
+        bulk_load(buf + m->run_off[q] + static_cast<long long>(k) * m->run_w[q],
+                  a.part_o + (slot * a.H + m->run_h[q]) * a.d + m->run_d0[q],
+                  static_cast<uint32_t>(m->run_w[q]) * 4u, &m->merge_bar);
+      }
+      // ---- split weights: one warp per run
+      for (int q = warp; q < nr; q += NWARPS) {
+        const int n = m->run_n[q], b = m->run_b[q], h = m->run_h[q], clo = m->run_clo[q];
+        float* w = buf + m->run_off[q] + static_cast<long long>(n) * m->run_w[q];
+        float mx = -INFINITY;
+        for (int k = lane; k < n; k += 32) {
+          const long long c = clo + k;
+          const float mk =
+              cta_empty(c, U, G) ? -INFINITY : __ldcg(a.part_ml + ((c + b) * a.H + h) * 2);
+          w[k] = mk;
+          mx = fmaxf(mx, mk);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float ls = 0.f;
+        for (int k = lane; k < n; k += 32) {
+          const long long c = clo + k;
+          const float mk = w[k];
+          const float wk = mk == -INFINITY ? 0.f : exp2f(mk - mx);
+          if (wk != 0.f) ls += wk * __ldcg(a.part_ml + ((c + b) * a.H + h) * 2 + 1);
+          w[k] = wk;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+        if (lane == 0) m->run_inv[q] = ls > 0.f ? 1.f / ls : 0.f;
+      }
+      bool ok = true;
+      if (m->group_bytes > 0) ok = mbar_wait(&m->merge_bar, phase, nullptr);
+      ok = __syncthreads_and(ok) != 0;
+      if (m->group_bytes > 0) phase ^= 1u;
+      if (!ok) {
+        failed = true;
+        if (tid == 0) set_err(a.err, LSA_DEVERR_TIMEOUT);
+        break;
+      }
+      // ---- outputs: one thread per (run, dimension)
+      int total_dims = 0;
+      for (int q = 0; q < nr; ++q) total_dims += m->run_w[q];
+      for (int t = tid; t < total_dims; t += NTHREADS) {
+        int q = 0, x = t;
+        while (x >= m->run_w[q]) x -= m->run_w[q++];
+        const int n = m->run_n[q], wq = m->run_w[q];
+        const float* rows = buf + m->run_off[q];
+        const float* w = rows + static_cast<long long>(n) * wq;
+        float acc = 0.f;
+        for (int k = 0; k < n; ++k) {
+          const float wk = w[k];
+          if (wk != 0.f) acc += wk * rows[static_cast<long long>(k) * wq + x];
+        }
+        const __nv_bfloat16 v = __float2bfloat16_rn(acc * m->run_inv[q]);
+        a.out[(static_cast<long long>(m->run_b[q]) * a.H + m->run_h[q]) * a.d + m->run_d0[q] + x] =
+            *reinterpret_cast<const uint16_t*>(&v);
+      }
+      __syncthreads();                  // the buffer is refilled by the next group
     }
+    if (nrec < MAXITEMS) break;
   }
   // ---- departure: the last CTA out resets the counters for the next launch
   __syncthreads();
@@ -816,6 +874,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // a sequence held whole by this CTA is normalised and written out here; a split
         // one leaves its partial (O, m, l) in slot CTA + sequence for the merge
         const bool whole = sg.u0 == 0 && sg.u1 == seq_units(a, sg.b);
+        // the CTA's last segment: Q and the ring are idle, so the result is staged there
+        // and written with one bulk copy instead of per-thread scalar stores
+        const bool staged = g == nseg - 1 && !m->more;
         const long long slot = static_cast<long long>(blockIdx.x) + sg.b;
         if (t128 < a.H) {
           const int h = t128;
@@ -830,6 +891,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (whole) named_bar_sync(1, 128);
         float* po = a.part_o + slot * a.H * a.d;
         uint16_t* fo = a.out + static_cast<long long>(sg.b) * a.H * a.d;
+        float* stf = reinterpret_cast<float*>(smem);
+        uint16_t* stb = reinterpret_cast<uint16_t*>(smem);
 #pragma unroll
         for (int db = 0; db < NDB; ++db) {
 #pragma unroll
@@ -844,12 +907,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const long long idx = static_cast<long long>(h) * a.d + db * 128 + row;
                 if (whole) {
                   const __nv_bfloat16 v = __float2bfloat16_rn(o[i] * m->alpha[h]);
-                  fo[idx] = *reinterpret_cast<const uint16_t*>(&v);
+                  (staged ? stb : fo)[idx] = *reinterpret_cast<const uint16_t*>(&v);
                 } else {
-                  po[idx] = o[i];
+                  (staged ? stf : po)[idx] = o[i];
                 }
               }
             }
+          }
+        }
+        if (staged) {
+          fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (t128 == 0) {
+            if (whole)
+              bulk_store(fo, stb, static_cast<uint32_t>(a.H) * a.d * 2);
+            else
+              bulk_store(po, stf, static_cast<uint32_t>(a.H) * a.d * 4);
+            bulk_commit_and_wait();
+            fence_proxy_async_global();
           }
         }
         tc_fence_before();
@@ -891,7 +966,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __shared__ long long s_U;
     if (tid == 0) s_U = U;
     __syncthreads();
-    merge_phase(a, m, reinterpret_cast<float*>(smem), s_U, *abort != 0);
+    merge_phase(a, m, reinterpret_cast<float*>(smem), LY::MISC_OFF / 4, s_U, *abort != 0);
   }
 }
 
@@ -981,7 +1056,7 @@ lsa_status decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pa
   if (append && ((reinterpret_cast<uintptr_t>(append->k_new) |
                   reinterpret_cast<uintptr_t>(append->v_new)) & 15u))
     return LSA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(out) & 1u) != 0) return LSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(out) & 15u) != 0) return LSA_ERR_INVALID_ARG;
   const int G = sm_count();
   if (G <= 0) return LSA_ERR_CUDA;
   if (G > lsa::attn::MAX_GRID) return LSA_ERR_UNIMPLEMENTED;
