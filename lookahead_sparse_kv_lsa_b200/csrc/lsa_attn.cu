@@ -404,12 +404,15 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
           if (run_end > hi) run_end = hi;
           int nchunks = static_cast<int>(run_end - j);
           const int n = m->item_chi[r] - m->item_clo[r] + 1;   // 0: empty sequence
-          long long need = static_cast<long long>(n) * (nchunks * 64) + n;
+          // rows, then the n weights padded to 4 floats so that every run's rows start
+          // on a 16-byte boundary (bulk copies require it)
+          const int wpad = (n + 3) & ~3;
+          long long need = static_cast<long long>(n) * (nchunks * 64) + wpad;
           if (used + need > buf_floats) {
             if (nr > 0) break;
-            nchunks = static_cast<int>((buf_floats / (n > 0 ? n : 1) - 1) / 64);
-            if (nchunks < 1) nchunks = 1;  // buf_floats >= 256 * 65 by construction
-            need = static_cast<long long>(n) * (nchunks * 64) + n;
+            nchunks = static_cast<int>((buf_floats - wpad) / (n > 0 ? n : 1) / 64);
+            if (nchunks < 1) nchunks = 1;  // buf_floats >= 256 * 64 + 256 by construction
+            need = static_cast<long long>(n) * (nchunks * 64) + wpad;
           }
           m->run_b[nr] = m->item_b[r];
           m->run_h[nr] = h;
