@@ -231,6 +231,7 @@ __device__ __noinline__ void plan_merge(const Args& a, long long U, int skip, Mi
     for (int b0 = 0; b0 < a.B; b0 += 32) {
       const int b = b0 + lane;
       const int u = b < a.B ? seq_units(a, b) : 0;
+      if (b < a.B && b % G == cta && seq_malformed(a, b)) set_err(a.err, LSA_DEVERR_BAD_SIZE);
       long long incl = u;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -255,7 +256,6 @@ __device__ __noinline__ void plan_merge(const Args& a, long long U, int skip, Mi
   for (int b0 = 0; b0 < a.B && base_i < j1; b0 += 32) {
     const int b = b0 + lane;
     const int u = b < a.B ? seq_units(a, b) : 0;
-    if (b < a.B && b % G == cta && seq_malformed(a, b)) set_err(a.err, LSA_DEVERR_BAD_SIZE);
     long long incl = u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -896,13 +896,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint16_t* fo = a.out + static_cast<long long>(sg.b) * a.H * a.d;
         float* stf = reinterpret_cast<float*>(smem);
         uint16_t* stb = reinterpret_cast<uint16_t*>(smem);
-#pragma unroll
+#pragma unroll 1
         for (int db = 0; db < NDB; ++db) {
+          float ob[HP];
+          tmem_ld_row<HP>(tmem + lane_addr + 2 * HP + db * HP, ob);
+          tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < HP / 16; ++c) {
-            float o[16];
-            tmem_ld16(tmem + lane_addr + 2 * HP + db * HP + 16 * c, o);
-            tmem_wait_ld();
+            const float* o = ob + 16 * c;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int h = 16 * c + i;
