@@ -901,22 +901,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           float ob[HP];
           tmem_ld_row<HP>(tmem + lane_addr + 2 * HP + db * HP, ob);
           tmem_wait_ld();
+          const int col = db * 128 + row;       // this thread's head-dimension index
+          if (staged) {
+            // [H][d] image in shared memory: lanes write consecutive words (no conflicts)
+            if (whole) {
+              const uint32_t base = smem_u32(stb) + col * 2;
 #pragma unroll
-          for (int c = 0; c < HP / 16; ++c) {
-            const float* o = ob + 16 * c;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int h = 16 * c + i;
-              if (h < a.H) {
-                const long long idx = static_cast<long long>(h) * a.d + db * 128 + row;
-                if (whole) {
-                  const __nv_bfloat16 v = __float2bfloat16_rn(o[i] * m->alpha[h]);
-                  (staged ? stb : fo)[idx] = *reinterpret_cast<const uint16_t*>(&v);
-                } else {
-                  (staged ? stf : po)[idx] = o[i];
+              for (int h = 0; h < HP; ++h)
+                if (h < a.H) {
+                  const __nv_bfloat16 v = __float2bfloat16_rn(ob[h] * m->alpha[h]);
+                  st_shared_u16(base + h * a.d * 2, *reinterpret_cast<const uint16_t*>(&v));
                 }
-              }
+            } else {
+              const uint32_t base = smem_u32(stf) + col * 4;
+#pragma unroll
+              for (int h = 0; h < HP; ++h)
+                if (h < a.H) st_shared_f32(base + h * a.d * 4, ob[h]);
             }
+          } else if (whole) {
+#pragma unroll
+            for (int h = 0; h < HP; ++h)
+              if (h < a.H) {
+                const __nv_bfloat16 v = __float2bfloat16_rn(ob[h] * m->alpha[h]);
+                fo[static_cast<long long>(h) * a.d + col] = *reinterpret_cast<const uint16_t*>(&v);
+              }
+          } else {
+#pragma unroll
+            for (int h = 0; h < HP; ++h)
+              if (h < a.H) po[static_cast<long long>(h) * a.d + col] = ob[h];
           }
         }
         if (staged) {

@@ -169,6 +169,15 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
   return v;
 }
 
+// Plain shared stores (volatile: kept in order with the fences and barriers that
+// follow them; no memory clobber, so surrounding loads may still be scheduled freely).
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v));
+}
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v));
+}
+
 // Order this thread's generic-proxy shared-memory writes before later async-proxy
 // (tensor core / TMA) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {
