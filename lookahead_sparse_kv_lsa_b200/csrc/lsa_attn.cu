@@ -160,6 +160,22 @@ __device__ __noinline__ void plan_segments(const Args& a, long long us, long lon
   }
 }
 
+// Units [tu0, tu1) of tile t of a segment. The segment's partial tile (fewer than 4
+// units) comes first: its small loads overlap the pipeline fill, and the segment ends on
+// full tiles, so a CTA with one unit more than another does not pay an extra round trip
+// at the end.
+__device__ __forceinline__ void tile_range(const Seg& sg, int t, int& tu0, int& tu1) {
+  const int len = sg.u1 - sg.u0;
+  const int first = (len & 3) ? (len & 3) : 4;
+  if (t == 0) {
+    tu0 = sg.u0;
+    tu1 = sg.u0 + (first < len ? first : len);
+  } else {
+    tu0 = sg.u0 + first + 4 * (t - 1);
+    tu1 = tu0 + 4 < sg.u1 ? tu0 + 4 : sg.u1;
+  }
+}
+
 // Butterfly reduce-scatter over the 32 lanes of a warp: afterwards lane l holds the
 // reduction of heads [l*N/32, l*N/32 + N/32) in v[0..] (N >= 32), or of head l/2 (N == 16).
 template <int N, bool IS_MAX>
@@ -452,27 +468,33 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
                   a.part_o + (slot * a.H + m->run_h[q]) * a.d + m->run_d0[q],
                   static_cast<uint32_t>(m->run_w[q]) * 4u, &m->merge_bar);
       }
-      // ---- split weights: one warp per run
+      // ---- split weights: one warp per run; all (m, l) pairs of a run are loaded in
+      // one batch (up to MAX_GRID / 32 per lane) so the weights cost one round trip
       for (int q = warp; q < nr; q += NWARPS) {
         const int n = m->run_n[q], b = m->run_b[q], h = m->run_h[q], clo = m->run_clo[q];
         float* w = buf + m->run_off[q] + static_cast<long long>(n) * m->run_w[q];
-        float mx = -INFINITY;
-        for (int k = lane; k < n; k += 32) {
+        constexpr int PER_LANE = MAX_GRID / 32;
+        float2 ml[PER_LANE];
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) {
+          const int k = lane + 32 * i;
           const long long c = clo + k;
-          const float mk =
-              cta_empty(c, U, G) ? -INFINITY : __ldcg(a.part_ml + ((c + b) * a.H + h) * 2);
-          w[k] = mk;
-          mx = fmaxf(mx, mk);
+          ml[i] = make_float2(-INFINITY, 0.f);
+          if (k < n && !cta_empty(c, U, G))
+            ml[i] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (c + b) * a.H + h);
         }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) mx = fmaxf(mx, ml[i].x);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float ls = 0.f;
-        for (int k = lane; k < n; k += 32) {
-          const long long c = clo + k;
-          const float mk = w[k];
-          const float wk = mk == -INFINITY ? 0.f : exp2f(mk - mx);
-          if (wk != 0.f) ls += wk * __ldcg(a.part_ml + ((c + b) * a.H + h) * 2 + 1);
-          w[k] = wk;
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) {
+          const int k = lane + 32 * i;
+          const float wk = ml[i].x == -INFINITY ? 0.f : exp2f(ml[i].x - mx);
+          ls += wk * ml[i].y;
+          if (k < n) w[k] = wk;
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
@@ -645,8 +667,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               // stage order per step i: K of tile i, then V of tile i-1
               const int tile = kv == 0 ? i : i - 1;
               if (tile < 0 || tile >= T) continue;
-              const int tu0 = sg.u0 + 4 * tile;
-              const int tu1 = min(tu0 + 4, sg.u1);
+              int tu0, tu1;
+              tile_range(sg, tile, tu0, tu1);
               int ys[4];
 #pragma unroll
               for (int r = 0; r < 4; ++r) {
@@ -775,8 +797,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(&m->s_full[sb], (gtile_s >> 1) & 1, abort));
           tc_fence_after();
           // validity of this row's token
-          const int u = sg.u0 + 4 * j + sw;
-          bool valid = u < sg.u1;
+          int tu0, tu1;
+          tile_range(sg, j, tu0, tu1);
+          const int u = tu0 + sw;
+          bool valid = u < tu1;
           if (valid && (u >> 1) == n_ent - 1) valid = (u & 1) * UNIT + lane < tl;
           // per-head tile max
           if (!failed) {
