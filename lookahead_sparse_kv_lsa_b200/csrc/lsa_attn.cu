@@ -66,6 +66,7 @@ struct Misc {
   int run_b[MAXRUNS], run_h[MAXRUNS], run_d0[MAXRUNS], run_w[MAXRUNS], run_clo[MAXRUNS],
       run_n[MAXRUNS], run_off[MAXRUNS];
   float run_inv[MAXRUNS];
+  long long ustart[MAX_GRID + 1];   // first unit of each CTA: floor(c * U / G)
 };
 
 struct Args {
@@ -358,6 +359,7 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
   constexpr int NWARPS = NTHREADS / 32;
   const long long G = gridDim.x;
   const int nch = a.d / 64;
+  for (int c = tid; c <= G; c += NTHREADS) m->ustart[c] = (static_cast<long long>(c) * U) / G;
   if (warp == 0) plan_merge(a, U, 0, m, lane);
   __syncthreads();
   if (m->total_items == 0) return;     // nothing split or empty: no barrier, all CTAs agree
@@ -480,7 +482,7 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
           const int k = lane + 32 * i;
           const long long c = clo + k;
           ml[i] = make_float2(-INFINITY, 0.f);
-          if (k < n && !cta_empty(c, U, G))
+          if (k < n && m->ustart[c] != m->ustart[c + 1])
             ml[i] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (c + b) * a.H + h);
         }
         float mx = -INFINITY;
@@ -518,11 +520,24 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
         const int n = m->run_n[q], wq = m->run_w[q];
         const float* rows = buf + m->run_off[q];
         const float* w = rows + static_cast<long long>(n) * wq;
-        float acc = 0.f;
-        for (int k = 0; k < n; ++k) {
-          const float wk = w[k];
-          if (wk != 0.f) acc += wk * rows[static_cast<long long>(k) * wq + x];
+        // 8 independent partial sums keep 8 shared loads in flight (zero weights mark
+        // empty CTAs, whose rows were copied but are never used)
+        float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        int k = 0;
+        for (; k + 8 <= n; k += 8) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float wk = w[k + i];
+            const float r = rows[static_cast<long long>(k + i) * wq + x];
+            acc8[i] += wk != 0.f ? wk * r : 0.f;
+          }
         }
+        for (; k < n; ++k) {
+          const float wk = w[k];
+          acc8[0] += wk != 0.f ? wk * rows[static_cast<long long>(k) * wq + x] : 0.f;
+        }
+        const float acc = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) +
+                          ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
         const __nv_bfloat16 v = __float2bfloat16_rn(acc * m->run_inv[q]);
         a.out[(static_cast<long long>(m->run_b[q]) * a.H + m->run_h[q]) * a.d + m->run_d0[q] + x] =
             *reinterpret_cast<const uint16_t*>(&v);
