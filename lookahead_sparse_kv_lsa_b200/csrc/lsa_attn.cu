@@ -40,6 +40,7 @@ constexpr int MAXSEG = 16;                // segments planned per batch
 constexpr float RESCALE_LOG2 = 8.0f;      // raise the running max only by more than 2^8
 constexpr int MAXITEMS = 64;              // sequences a CTA's merge range meets, per round
 constexpr int MAXRUNS = 32;               // (sequence, head, chunk range) runs per merge group
+constexpr int SCRATCH_FLOATS = 4 * NTHREADS;  // merge scratch after a group's rows
 constexpr int MAX_GRID = 256;             // CTAs per launch (one per SM)
 
 struct Seg {
@@ -353,23 +354,22 @@ __device__ __forceinline__ float block_sum(float v, Misc* m, int tid, int nwarps
 // fits the idle shared memory has all its partial rows fetched with 1-D bulk copies
 // (issued by all threads, one round trip) while one warp per run derives the split
 // weights; then every thread reduces a few output dimensions over the partials.
-__device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int buf_floats,
+__device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, int buf_floats,
                                          long long U, bool aborted) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NWARPS = NTHREADS / 32;
   const long long G = gridDim.x;
   const int nch = a.d / 64;
-  for (int c = tid; c <= G; c += NTHREADS) m->ustart[c] = (static_cast<long long>(c) * U) / G;
-  if (warp == 0) plan_merge(a, U, 0, m, lane);
-  __syncthreads();
+  // m->ustart and the round-0 plan were filled by the producer warp after its last loads
   if (m->total_items == 0) return;     // nothing split or empty: no barrier, all CTAs agree
   // ---- grid barrier: all partials written before any is read
   if (tid == 0) {
     __threadfence();
-    atomicAdd(a.sync, 1u);
+    const unsigned int before = atomicAdd(a.sync, 1u);
     const uint64_t t0 = globaltimer_ns();
     bool ok = true;
-    while (ld_acquire_gpu(a.sync) < static_cast<unsigned int>(G)) {
+    while (before + 1u < static_cast<unsigned int>(G) &&
+           ld_acquire_gpu(a.sync) < static_cast<unsigned int>(G)) {
       __nanosleep(32);
       if (globaltimer_ns() - t0 > LSA_WAIT_LIMIT_NS) {
         ok = false;
@@ -386,6 +386,7 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
   __syncthreads();
   bool failed = m->abort != 0 || aborted;   // the same value in every thread
   uint32_t phase = 0;
+  bool first_group = true;   // the epilogue fenced its own shared writes before this
   for (int round = 0; !failed; ++round) {
     if (round > 0) {
       __syncthreads();
@@ -416,8 +417,9 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
             j = -1;
             continue;
           }
-          const int h = static_cast<int>((j - ib) / nch);
-          const int c0 = static_cast<int>((j - ib) % nch);
+          const int rel = static_cast<int>(j - ib);   // < H * nch: 32-bit division
+          const int h = rel / nch;
+          const int c0 = rel - h * nch;
           long long run_end = ib + static_cast<long long>(h + 1) * nch;
           if (run_end > hi) run_end = hi;
           int nchunks = static_cast<int>(run_end - j);
@@ -426,9 +428,9 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
           // on a 16-byte boundary (bulk copies require it)
           const int wpad = (n + 3) & ~3;
           long long need = static_cast<long long>(n) * (nchunks * 64) + wpad;
-          if (used + need > buf_floats) {
+          if (used + need > buf_floats - SCRATCH_FLOATS) {
             if (nr > 0) break;
-            nchunks = static_cast<int>((buf_floats - wpad) / (n > 0 ? n : 1) / 64);
+            nchunks = static_cast<int>((buf_floats - SCRATCH_FLOATS - wpad) / (n > 0 ? n : 1) / 64);
             if (nchunks < 1) nchunks = 1;  // buf_floats >= 256 * 64 + 256 by construction
             need = static_cast<long long>(n) * (nchunks * 64) + wpad;
           }
@@ -461,7 +463,8 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
       // ---- partial rows: one bulk copy per (run, split), spread over all threads
       int total_rows = 0;
       for (int q = 0; q < nr; ++q) total_rows += m->run_n[q];
-      fence_proxy_async_smem();         // this thread's earlier reads of the buffer first
+      if (!first_group) fence_proxy_async_smem();   // this thread's reads of the last group
+      first_group = false;
       for (int t = tid; t < total_rows; t += NTHREADS) {
         int q = 0, k = t;
         while (k >= m->run_n[q]) k -= m->run_n[q++];
@@ -511,36 +514,61 @@ __device__ __noinline__ void merge_phase(const Args& a, Misc* m, float* buf, int
         if (tid == 0) set_err(a.err, LSA_DEVERR_TIMEOUT);
         break;
       }
-      // ---- outputs: one thread per (run, dimension)
-      int total_dims = 0;
-      for (int q = 0; q < nr; ++q) total_dims += m->run_w[q];
-      for (int t = tid; t < total_dims; t += NTHREADS) {
-        int q = 0, x = t;
-        while (x >= m->run_w[q]) x -= m->run_w[q++];
-        const int n = m->run_n[q], wq = m->run_w[q];
-        const float* rows = buf + m->run_off[q];
-        const float* w = rows + static_cast<long long>(n) * wq;
-        // 8 independent partial sums keep 8 shared loads in flight (zero weights mark
-        // empty CTAs, whose rows were copied but are never used)
-        float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        int k = 0;
-        for (; k + 8 <= n; k += 8) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float wk = w[k + i];
-            const float r = rows[static_cast<long long>(k + i) * wq + x];
-            acc8[i] += wk != 0.f ? wk * r : 0.f;
+      // ---- outputs: threads take (run, 4-dim column, split slice) triples; each sums
+      // its slice of the splits with float4 shared loads, the slices meet in scratch
+      int total_c4 = 0;
+      for (int q = 0; q < nr; ++q) total_c4 += m->run_w[q] >> 2;
+      int slices = NTHREADS / (total_c4 > 0 ? total_c4 : 1);
+      slices = slices < 1 ? 1 : (slices > 8 ? 8 : slices);
+      float4* scratch = reinterpret_cast<float4*>(buf + m->group_floats);
+      for (int base = 0; base < total_c4; base += NTHREADS / slices) {
+        const int per = NTHREADS / slices;
+        const int t = tid / slices, sl = tid - t * slices;
+        const int c4 = base + t;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        int q = 0;
+        if (t < per && c4 < total_c4) {
+          int x = c4;
+          while (x >= (m->run_w[q] >> 2)) x -= m->run_w[q++] >> 2;
+          const int n = m->run_n[q], wq = m->run_w[q];
+          const float* rows = buf + m->run_off[q] + 4 * x;
+          const float* w = buf + m->run_off[q] + static_cast<long long>(n) * wq;
+#pragma unroll 4
+          for (int k = sl; k < n; k += slices) {
+            const float wk = w[k];
+            if (wk != 0.f) {              // zero weight: an empty CTA's (unused) row
+              const float4 r = *reinterpret_cast<const float4*>(rows + static_cast<long long>(k) * wq);
+              acc.x += wk * r.x;
+              acc.y += wk * r.y;
+              acc.z += wk * r.z;
+              acc.w += wk * r.w;
+            }
           }
         }
-        for (; k < n; ++k) {
-          const float wk = w[k];
-          acc8[0] += wk != 0.f ? wk * rows[static_cast<long long>(k) * wq + x] : 0.f;
+        scratch[tid] = acc;
+        __syncthreads();
+        if (sl == 0 && t < per && c4 < total_c4) {
+          float4 tot = scratch[tid];
+          for (int j = 1; j < slices; ++j) {
+            const float4 v = scratch[tid + j];
+            tot.x += v.x;
+            tot.y += v.y;
+            tot.z += v.z;
+            tot.w += v.w;
+          }
+          int x = c4;
+          q = 0;
+          while (x >= (m->run_w[q] >> 2)) x -= m->run_w[q++] >> 2;
+          const float inv = m->run_inv[q];
+          const __nv_bfloat162 p0 = __floats2bfloat162_rn(tot.x * inv, tot.y * inv);
+          const __nv_bfloat162 p1 = __floats2bfloat162_rn(tot.z * inv, tot.w * inv);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t*>(&p0);
+          pk.y = *reinterpret_cast<const uint32_t*>(&p1);
+          *reinterpret_cast<uint2*>(a.out + (static_cast<long long>(m->run_b[q]) * a.H + m->run_h[q]) *
+                                                a.d + m->run_d0[q] + 4 * x) = pk;
         }
-        const float acc = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) +
-                          ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
-        const __nv_bfloat16 v = __float2bfloat16_rn(acc * m->run_inv[q]);
-        a.out[(static_cast<long long>(m->run_b[q]) * a.H + m->run_h[q]) * a.d + m->run_d0[q] + x] =
-            *reinterpret_cast<const uint16_t*>(&v);
+        __syncthreads();
       }
       __syncthreads();                  // the buffer is refilled by the next group
     }
@@ -712,6 +740,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
           }
         }
+      }
+      __syncwarp();
+      if (!m->more) {
+        // the producer's last loads are out: plan the fused merge meanwhile
+        for (int c = lane; c <= G; c += 32) m->ustart[c] = (c * U) / G;
+        plan_merge(a, U, 0, m, lane);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------- MMA issuer
