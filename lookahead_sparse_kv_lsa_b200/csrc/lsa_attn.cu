@@ -610,8 +610,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   using LY = Layout<HP, NDC>;
   constexpr int NDB = LY::NDB;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, derived by pointer arithmetic on the shared array so the
+  // compiler keeps addressing it as shared memory (no generic loads and stores)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem + LY::Q_OFF;
   uint8_t* sRing = smem + LY::RING_OFF;
   uint8_t* sP = smem + LY::P_OFF;
