@@ -338,7 +338,7 @@ def oracle_pass_seconds(wl, steps):
     return t_idx + c.tau * per_step, time.perf_counter() - t_start
 
 
-def cpu_baseline(wl, steps=tuple(range(0, 64, 3))):
+def cpu_baseline(wl, steps=tuple(range(64))):
     c = wl.cfg
     t_pass, spent = oracle_pass_seconds(wl, steps)
     return {"value": c.B * c.tau / t_pass, "unit": UNIT, "cores": oracle_threads(),
