@@ -161,6 +161,33 @@ lsa_status lsa_decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t 
 size_t lsa_decode_attn_workspace_size(int32_t B, int32_t H, int32_t d, int32_t n_sm);
 
 /* ---------------------------------------------------------------------------------
+ * lsa_decode_attn_noalloc -- lsa_decode_attn for callers that cannot allocate device
+ * memory (no counterpart on the pages: it is a deployment convenience). Some callers
+ * run inside a host framework that owns every allocation, or in a loop that must never
+ * enter the CUDA allocator, or receive only their input and output buffers; they
+ * cannot provide the workspace lsa_decode_attn needs for its split partials.
+ *
+ * This entry point takes the same arguments minus the workspace and uses instead one
+ * fixed device array inside this library, LSA_NOALLOC_SCRATCH_BYTES large, which every
+ * GPU that loads the library holds until the process exits. The call allocates nothing
+ * (no cudaMalloc, cudaFree or allocating library routine).
+ *  - Limit: lsa_decode_attn_workspace_size(B, H, d, n_sm) must not exceed
+ *    LSA_NOALLOC_SCRATCH_BYTES (e.g. B <= 107 at H = 64, d = 512, 148 SMs); larger
+ *    problems return LSA_ERR_CAPACITY before anything is enqueued.
+ *  - The first call on a device looks up the array's device address and zeroes it
+ *    (synchronously); make that first call before any stream capture.
+ *  - Every call shares the array: calls that overlap on the GPU (other streams,
+ *    other host threads) race and produce wrong results. Serialise them.
+ *  - The caller still provides and owns q, the pool, the block table, out and err.
+ */
+#define LSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+lsa_status lsa_decode_attn_noalloc(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pages,
+                                   const int32_t* block_table, int32_t bt_stride,
+                                   const int32_t* n_entries, const int32_t* tail_len,
+                                   int32_t B, int32_t H, int32_t d, float scale,
+                                   uint16_t* out, int32_t* err, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * lsa_step -- the decode loop of section 2 (steps 1-5) for a batch of B sequences.
  *
  * Pass p covers global decode steps 64p .. 64p+63. When it starts, sequence b holds

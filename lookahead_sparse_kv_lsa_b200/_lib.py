@@ -58,6 +58,8 @@ SIGNATURES = {
     "lsa_decode_attn": (_i32, [_p, _p, _i64, _p, _i32, _p, _p, _i32, _i32, _i32, C.c_float, _p,
                                _p, _sz, _p, _p]),
     "lsa_decode_attn_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
+    "lsa_decode_attn_noalloc": (_i32, [_p, _p, _i64, _p, _i32, _p, _p, _i32, _i32, _i32,
+                                       C.c_float, _p, _p, _p]),
     "lsa_state_check": (_i32, [C.POINTER(LsaState)]),
     "lsa_state_size": (_sz, []),
     "lsa_load_window": (_i32, [C.POINTER(LsaState), _i32, _p]),

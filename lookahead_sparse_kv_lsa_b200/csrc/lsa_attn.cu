@@ -28,6 +28,8 @@
 
 #include <math.h>
 
+#include <mutex>
+
 namespace lsa {
 namespace attn {
 
@@ -1208,4 +1210,67 @@ extern "C" lsa_status lsa_decode_attn(const uint16_t* q, const uint16_t* hbm_poo
                                       void* ws, size_t ws_bytes, int32_t* err, void* stream) {
   return lsa_host::decode_attn(q, hbm_pool, n_pages, block_table, bt_stride, n_entries, tail_len,
                                B, H, d, scale, out, ws, ws_bytes, err, stream, nullptr);
+}
+
+// ------------------------------------------------- decode attention without allocation
+// For callers that cannot allocate device memory at all, e.g. code running inside a
+// host framework that owns every allocation, a real-time loop that must not call into
+// the CUDA allocator, or a plugin that receives only input and output buffers: the split
+// partials and the merge barrier counters live in one fixed device array of this library.
+// Every call shares the array, so calls that overlap on the GPU race with one another.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LSA_NOALLOC_SCRATCH_BYTES];
+
+struct NoallocScratch {
+  void* ptr = nullptr;
+  bool ready = false;
+};
+
+std::mutex g_noalloc_mutex;
+NoallocScratch g_noalloc[64];
+
+// Device address of the scratch array on the current device. In host code the array's
+// name is only a host-side stand-in, so the address is queried once per device (with
+// that device current) and the barrier counters are zeroed then.
+lsa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  NoallocScratch& s = g_noalloc[dev];
+  if (!s.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return LSA_ERR_CUDA;
+    }
+    if (cudaMemset(p, 0, LSA_NOALLOC_SCRATCH_BYTES) != cudaSuccess) {
+      cudaGetLastError();
+      return LSA_ERR_CUDA;
+    }
+    s.ptr = p;
+    s.ready = true;
+  }
+  *out = s.ptr;
+  return LSA_OK;
+}
+
+}  // namespace
+
+extern "C" lsa_status lsa_decode_attn_noalloc(const uint16_t* q, const uint16_t* hbm_pool,
+                                              int64_t n_pages, const int32_t* block_table,
+                                              int32_t bt_stride, const int32_t* n_entries,
+                                              const int32_t* tail_len, int32_t B, int32_t H,
+                                              int32_t d, float scale, uint16_t* out,
+                                              int32_t* err, void* stream) {
+  if (B <= 0 || H <= 0 || d <= 0) return LSA_ERR_INVALID_ARG;
+  const int G = lsa_host::sm_count();
+  if (G <= 0) return LSA_ERR_CUDA;
+  const size_t need = attn_ws_bytes(B, H, d, G);
+  if (need > static_cast<size_t>(LSA_NOALLOC_SCRATCH_BYTES)) return LSA_ERR_CAPACITY;
+  void* ws = nullptr;
+  const lsa_status st = noalloc_scratch(&ws);
+  if (st != LSA_OK) return st;
+  return lsa_host::decode_attn(q, hbm_pool, n_pages, block_table, bt_stride, n_entries, tail_len,
+                               B, H, d, scale, out, ws, need, err, stream, nullptr);
 }
