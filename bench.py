@@ -381,13 +381,23 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------- lsa arm
 def max_over_ranks(x, world):
+    """The largest of every rank's x (device time of the timed region): all ranks call
+    it at the same point with the same world size. Works on nccl (CUDA tensor) and
+    gloo (CPU tensor) process groups."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank, world, max_ms):
+    """Replicas: every rank decodes its own batch; the job rate is all ranks' tokens over
+    the slowest rank's time."""
+    return world * tokens_per_rank / (max_ms * 1e-3)
 
 
 def barrier(world):
@@ -520,9 +530,9 @@ def run_lsa(args, rank, world, local):
     gth_avg = statistics.mean(gth_ms)
     h2d_peak = pinned_h2d_gbs(dev)
 
-    tokens = world * cfg.B * cfg.tau * args.steps
     line = {
-        "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": whole_job_rate(cfg.B * cfg.tau * args.steps, world, ms),
+        "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
