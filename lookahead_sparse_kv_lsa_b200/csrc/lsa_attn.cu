@@ -52,7 +52,7 @@ struct Seg {
 struct Misc {
   uint64_t full[NST], empty[NST];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, q_full, q_free, mma_done, merge_bar;
+  uint64_t p_full, pv_done, q_full, q_free, mma_done;
   uint32_t tmem_base;
   int abort;
   int nseg, more;
@@ -64,7 +64,6 @@ struct Misc {
   int n_items, total_items;
   long long merge_j0, merge_j1, cur_j;
   int cur_rec, n_runs, group_floats;
-  uint32_t group_bytes;
   int item_b[MAXITEMS], item_h[MAXITEMS], item_clo[MAXITEMS], item_chi[MAXITEMS];
   int run_b[MAXRUNS], run_h[MAXRUNS], run_d0[MAXRUNS], run_w[MAXRUNS], run_clo[MAXRUNS],
       run_n[MAXRUNS], run_off[MAXRUNS];
@@ -387,8 +386,6 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
   }
   __syncthreads();
   bool failed = m->abort != 0 || aborted;   // the same value in every thread
-  uint32_t phase = 0;
-  bool first_group = true;   // the epilogue fenced its own shared writes before this
   for (int round = 0; !failed; ++round) {
     if (round > 0) {
       __syncthreads();
@@ -451,30 +448,29 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
         m->cur_j = j;
         m->n_runs = nr;
         m->group_floats = static_cast<int>(used);
-        uint32_t bytes = 0;
-        for (int q = 0; q < nr; ++q) bytes += static_cast<uint32_t>(m->run_n[q]) * m->run_w[q] * 4u;
-        m->group_bytes = bytes;
-        if (bytes > 0) {
-          fence_proxy_async_smem();     // earlier generic accesses of the buffer first
-          mbar_arrive_expect_tx(&m->merge_bar, bytes);
-        }
+
       }
       __syncthreads();
       const int nr = m->n_runs;
       if (nr == 0) break;
-      // ---- partial rows: one bulk copy per (run, split), spread over all threads
-      int total_rows = 0;
-      for (int q = 0; q < nr; ++q) total_rows += m->run_n[q];
-      if (!first_group) fence_proxy_async_smem();   // this thread's reads of the last group
-      first_group = false;
-      for (int t = tid; t < total_rows; t += NTHREADS) {
-        int q = 0, k = t;
-        while (k >= m->run_n[q]) k -= m->run_n[q++];
-        const long long slot = m->run_clo[q] + k + m->run_b[q];
-        bulk_load(buf + m->run_off[q] + static_cast<long long>(k) * m->run_w[q],
-                  a.part_o + (slot * a.H + m->run_h[q]) * a.d + m->run_d0[q],
-                  static_cast<uint32_t>(m->run_w[q]) * 4u, &m->merge_bar);
+      // ---- partial rows: 16-byte asynchronous copies from L2, spread over all threads
+      // (columns across threads, splits down the rows): one round trip for the group
+      for (int q = 0; q < nr; ++q) {
+        const int n = m->run_n[q], w4 = m->run_w[q] >> 2;
+        const int rows_per_pass = NTHREADS / w4;           // run_w <= 512: w4 <= 128
+        const int c = tid % w4, r0 = tid / w4;
+        if (r0 < rows_per_pass) {
+          const long long b = m->run_b[q], h = m->run_h[q];
+          const uint32_t dst0 = smem_u32(buf + m->run_off[q]) + c * 16;
+          const float* src0 = a.part_o + (h * a.d + m->run_d0[q] + 4 * c);
+          for (int k = r0; k < n; k += rows_per_pass) {
+            const long long slot = m->run_clo[q] + k + b;
+            cp_async16(dst0 + static_cast<uint32_t>(k) * (w4 * 16),
+                       src0 + slot * a.H * a.d);
+          }
+        }
       }
+      cp_async_commit();
       // ---- split weights: one warp per run; all (m, l) pairs of a run are loaded in
       // one batch (up to MAX_GRID / 32 per lane) so the weights cost one round trip
       for (int q = warp; q < nr; q += NWARPS) {
@@ -507,15 +503,8 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
         for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
         if (lane == 0) m->run_inv[q] = ls > 0.f ? 1.f / ls : 0.f;
       }
-      bool ok = true;
-      if (m->group_bytes > 0) ok = mbar_wait(&m->merge_bar, phase, nullptr);
-      ok = __syncthreads_and(ok) != 0;
-      if (m->group_bytes > 0) phase ^= 1u;
-      if (!ok) {
-        failed = true;
-        if (tid == 0) set_err(a.err, LSA_DEVERR_TIMEOUT);
-        break;
-      }
+      cp_async_wait_all();
+      __syncthreads();
       // ---- outputs: threads take (run, 4-dim column, split slice) triples; each sums
       // its slice of the splits with float4 shared loads, the slices meet in scratch
       int total_c4 = 0;
@@ -637,7 +626,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&m->q_full, 1);
     mbar_init(&m->q_free, 1);
     mbar_init(&m->mma_done, 1);
-    mbar_init(&m->merge_bar, 1);
     m->abort = 0;
     fence_barrier_init();
   }
@@ -970,8 +958,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (whole) named_bar_sync(1, 128);
         float* po = a.part_o + slot * a.H * a.d;
         uint16_t* fo = a.out + static_cast<long long>(sg.b) * a.H * a.d;
-        float* stf = reinterpret_cast<float*>(smem);
-        uint16_t* stb = reinterpret_cast<uint16_t*>(smem);
+        // staged: each 128-dim block is laid out [head][128] in its own region of the idle
+        // ring / Q buffers; right after a block is complete, one thread per head stores
+        // that head's row with a 1-D bulk copy, overlapping the staging of the next block
+        const int esz = whole ? 2 : 4;
+        const uint32_t blk_bytes = static_cast<uint32_t>(a.H) * 128u * esz;
+        bool issued = false;
 #pragma unroll 1
         for (int db = 0; db < NDB; ++db) {
           float ob[HP];
@@ -979,20 +971,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_wait_ld();
           const int col = db * 128 + row;       // this thread's head-dimension index
           if (staged) {
-            // [H][d] image in shared memory: lanes write consecutive words (no conflicts)
+            const uint32_t base = smem_u32(smem) + db * blk_bytes + row * esz;
             if (whole) {
-              const uint32_t base = smem_u32(stb) + col * 2;
 #pragma unroll
               for (int h = 0; h < HP; ++h)
                 if (h < a.H) {
                   const __nv_bfloat16 v = __float2bfloat16_rn(ob[h] * m->alpha[h]);
-                  st_shared_u16(base + h * a.d * 2, *reinterpret_cast<const uint16_t*>(&v));
+                  st_shared_u16(base + h * 256u, *reinterpret_cast<const uint16_t*>(&v));
                 }
             } else {
-              const uint32_t base = smem_u32(stf) + col * 4;
 #pragma unroll
               for (int h = 0; h < HP; ++h)
-                if (h < a.H) st_shared_f32(base + h * a.d * 4, ob[h]);
+                if (h < a.H) st_shared_f32(base + h * 512u, ob[h]);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (t128 < a.H) {
+              const uint8_t* src = smem + db * blk_bytes + t128 * 128 * esz;
+              if (whole)
+                bulk_store(fo + static_cast<long long>(t128) * a.d + db * 128, src, 256u);
+              else
+                bulk_store(po + static_cast<long long>(t128) * a.d + db * 128, src, 512u);
+              issued = true;
             }
           } else if (whole) {
 #pragma unroll
@@ -1007,17 +1007,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               if (h < a.H) po[static_cast<long long>(h) * a.d + col] = ob[h];
           }
         }
-        if (staged) {
-          fence_proxy_async_smem();
-          named_bar_sync(1, 128);
-          if (t128 == 0) {
-            if (whole)
-              bulk_store(fo, stb, static_cast<uint32_t>(a.H) * a.d * 2);
-            else
-              bulk_store(po, stf, static_cast<uint32_t>(a.H) * a.d * 4);
-            bulk_commit_and_wait();
-            fence_proxy_async_global();
-          }
+        if (issued) {
+          bulk_commit_and_wait();
+          fence_proxy_async_global();
         }
         tc_fence_before();
         named_bar_sync(1, 128);
