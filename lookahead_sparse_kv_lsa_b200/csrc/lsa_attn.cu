@@ -42,7 +42,7 @@ constexpr int MAXSEG = 16;                // segments planned per batch
 constexpr float RESCALE_LOG2 = 8.0f;      // raise the running max only by more than 2^8
 constexpr int MAXITEMS = 64;              // sequences a CTA's merge range meets, per round
 constexpr int MAXRUNS = 32;               // (sequence, head, chunk range) runs per merge group
-constexpr int SCRATCH_FLOATS = (NTHREADS / 32) * 64 * 8;  // merge scratch after a group's rows
+constexpr int SCRATCH_FLOATS = 4 * NTHREADS;  // merge scratch after a group's rows
 constexpr int MAX_GRID = 256;             // CTAs per launch (one per SM)
 
 struct Seg {
@@ -75,7 +75,7 @@ struct Args {
   const int32_t* block_table;
   const int32_t* n_entries;
   const int32_t* tail_len;
-  uint16_t* part_o;       // [slots][H][d] bf16, normalised partial O / l
+  float* part_o;          // [slots][H][d] fp32
   float* part_ml;         // [slots][H][2] fp32 (running max in log2 units, denominator)
   unsigned int* sync;     // [2] grid-barrier arrive / depart counters (left at zero)
   uint16_t* out;          // [B][H][d] bf16
@@ -425,15 +425,13 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
           const int n = m->item_chi[r] - m->item_clo[r] + 1;   // 0: empty sequence
           // rows, then the n weights padded to 4 floats so that every run's rows start
           // on a 16-byte boundary (bulk copies require it)
-          // rows: n x (nchunks * 64) bf16 = n * nchunks * 32 words; then the n weights
-          // padded to 4 words, so every run's rows start on a 16-byte boundary
           const int wpad = (n + 3) & ~3;
-          long long need = static_cast<long long>(n) * (nchunks * 32) + wpad;
+          long long need = static_cast<long long>(n) * (nchunks * 64) + wpad;
           if (used + need > buf_floats - SCRATCH_FLOATS) {
             if (nr > 0) break;
-            nchunks = static_cast<int>((buf_floats - SCRATCH_FLOATS - wpad) / (n > 0 ? n : 1) / 32);
-            if (nchunks < 1) nchunks = 1;  // buf_floats >= 256 * 32 + 256 + scratch
-            need = static_cast<long long>(n) * (nchunks * 32) + wpad;
+            nchunks = static_cast<int>((buf_floats - SCRATCH_FLOATS - wpad) / (n > 0 ? n : 1) / 64);
+            if (nchunks < 1) nchunks = 1;  // buf_floats >= 256 * 64 + 256 by construction
+            need = static_cast<long long>(n) * (nchunks * 64) + wpad;
           }
           m->run_b[nr] = m->item_b[r];
           m->run_h[nr] = h;
@@ -455,28 +453,29 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
       __syncthreads();
       const int nr = m->n_runs;
       if (nr == 0) break;
-      // ---- partial rows (bf16): 16-byte asynchronous copies from L2 spread over all
-      // threads (8-element columns across threads, splits down the rows): one round trip
+      // ---- partial rows: 16-byte asynchronous copies from L2, spread over all threads
+      // (columns across threads, splits down the rows): one round trip for the group
       for (int q = 0; q < nr; ++q) {
-        const int n = m->run_n[q], w8 = m->run_w[q] >> 3;
-        const int rows_per_pass = NTHREADS / w8;           // run_w <= 512: w8 <= 64
-        const int c = tid % w8, r0 = tid / w8;
+        const int n = m->run_n[q], w4 = m->run_w[q] >> 2;
+        const int rows_per_pass = NTHREADS / w4;           // run_w <= 512: w4 <= 128
+        const int c = tid % w4, r0 = tid / w4;
         if (r0 < rows_per_pass) {
           const long long b = m->run_b[q], h = m->run_h[q];
           const uint32_t dst0 = smem_u32(buf + m->run_off[q]) + c * 16;
-          const uint16_t* src0 = a.part_o + (h * a.d + m->run_d0[q] + 8 * c);
+          const float* src0 = a.part_o + (h * a.d + m->run_d0[q] + 4 * c);
           for (int k = r0; k < n; k += rows_per_pass) {
             const long long slot = m->run_clo[q] + k + b;
-            cp_async16(dst0 + static_cast<uint32_t>(k) * (w8 * 16), src0 + slot * a.H * a.d);
+            cp_async16(dst0 + static_cast<uint32_t>(k) * (w4 * 16),
+                       src0 + slot * a.H * a.d);
           }
         }
       }
       cp_async_commit();
-      // ---- split weights W_k = 2^(m_k - M) l_k (the rows are O_k / l_k): one warp per
-      // run, all (m, l) pairs of the run loaded in one batch
+      // ---- split weights: one warp per run; all (m, l) pairs of a run are loaded in
+      // one batch (up to MAX_GRID / 32 per lane) so the weights cost one round trip
       for (int q = warp; q < nr; q += NWARPS) {
         const int n = m->run_n[q], b = m->run_b[q], h = m->run_h[q], clo = m->run_clo[q];
-        float* w = buf + m->run_off[q] + static_cast<long long>(n) * (m->run_w[q] >> 1);
+        float* w = buf + m->run_off[q] + static_cast<long long>(n) * m->run_w[q];
         constexpr int PER_LANE = MAX_GRID / 32;
         float2 ml[PER_LANE];
 #pragma unroll
@@ -496,8 +495,8 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
 #pragma unroll
         for (int i = 0; i < PER_LANE; ++i) {
           const int k = lane + 32 * i;
-          const float wk = ml[i].x == -INFINITY ? 0.f : exp2f(ml[i].x - mx) * ml[i].y;
-          ls += wk;
+          const float wk = ml[i].x == -INFINITY ? 0.f : exp2f(ml[i].x - mx);
+          ls += wk * ml[i].y;
           if (k < n) w[k] = wk;
         }
 #pragma unroll
@@ -506,50 +505,59 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
       }
       cp_async_wait_all();
       __syncthreads();
-      // ---- outputs, one run at a time: lanes over 8-element columns (conflict-free
-      // 16-byte shared loads), warps over slices of the splits, slices summed in scratch
-      float* scratch = buf + m->group_floats;
-      for (int q = 0; q < nr; ++q) {
-        const int n = m->run_n[q], w8 = m->run_w[q] >> 3;
-        const int groups = (w8 + 31) >> 5;                 // 1 or 2
-        const int slices = NWARPS / groups;
-        const int cg = warp % groups, sl = warp / groups;
-        const int c = cg * 32 + lane;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (sl < slices && c < w8) {
-          const uint8_t* rows = reinterpret_cast<const uint8_t*>(buf + m->run_off[q]) + c * 16;
-          const float* w = buf + m->run_off[q] + static_cast<long long>(n) * (m->run_w[q] >> 1);
+      // ---- outputs: threads take (run, 4-dim column, split slice) triples; each sums
+      // its slice of the splits with float4 shared loads, the slices meet in scratch
+      int total_c4 = 0;
+      for (int q = 0; q < nr; ++q) total_c4 += m->run_w[q] >> 2;
+      int slices = NTHREADS / (total_c4 > 0 ? total_c4 : 1);
+      slices = slices < 1 ? 1 : (slices > 8 ? 8 : slices);
+      float4* scratch = reinterpret_cast<float4*>(buf + m->group_floats);
+      for (int base = 0; base < total_c4; base += NTHREADS / slices) {
+        const int per = NTHREADS / slices;
+        const int t = tid / slices, sl = tid - t * slices;
+        const int c4 = base + t;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        int q = 0;
+        if (t < per && c4 < total_c4) {
+          int x = c4;
+          while (x >= (m->run_w[q] >> 2)) x -= m->run_w[q++] >> 2;
+          const int n = m->run_n[q], wq = m->run_w[q];
+          const float* rows = buf + m->run_off[q] + 4 * x;
+          const float* w = buf + m->run_off[q] + static_cast<long long>(n) * wq;
 #pragma unroll 4
           for (int k = sl; k < n; k += slices) {
             const float wk = w[k];
-            const uint4 v = *reinterpret_cast<const uint4*>(rows + static_cast<long long>(k) * (w8 * 16));
-            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              // a zero weight marks an empty CTA's row, which is never read arithmetically
-              acc[2 * e] += wk != 0.f ? wk * __uint_as_float(vv[e] << 16) : 0.f;
-              acc[2 * e + 1] += wk != 0.f ? wk * __uint_as_float(vv[e] & 0xFFFF0000u) : 0.f;
+            if (wk != 0.f) {              // zero weight: an empty CTA's (unused) row
+              const float4 r = *reinterpret_cast<const float4*>(rows + static_cast<long long>(k) * wq);
+              acc.x += wk * r.x;
+              acc.y += wk * r.y;
+              acc.z += wk * r.z;
+              acc.w += wk * r.w;
             }
           }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) scratch[(sl * w8 + c) * 8 + e] = acc[e];
         }
+        scratch[tid] = acc;
         __syncthreads();
-        for (int t = tid; t < w8; t += NTHREADS) {
-          float tot[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          for (int j = 0; j < slices; ++j)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) tot[e] += scratch[(j * w8 + t) * 8 + e];
-          const float inv = m->run_inv[q];
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 p2 = __floats2bfloat162_rn(tot[2 * e] * inv, tot[2 * e + 1] * inv);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&p2);
+        if (sl == 0 && t < per && c4 < total_c4) {
+          float4 tot = scratch[tid];
+          for (int j = 1; j < slices; ++j) {
+            const float4 v = scratch[tid + j];
+            tot.x += v.x;
+            tot.y += v.y;
+            tot.z += v.z;
+            tot.w += v.w;
           }
-          *reinterpret_cast<uint4*>(a.out + (static_cast<long long>(m->run_b[q]) * a.H + m->run_h[q]) *
-                                                a.d + m->run_d0[q] + 8 * t) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          int x = c4;
+          q = 0;
+          while (x >= (m->run_w[q] >> 2)) x -= m->run_w[q++] >> 2;
+          const float inv = m->run_inv[q];
+          const __nv_bfloat162 p0 = __floats2bfloat162_rn(tot.x * inv, tot.y * inv);
+          const __nv_bfloat162 p1 = __floats2bfloat162_rn(tot.z * inv, tot.w * inv);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t*>(&p0);
+          pk.y = *reinterpret_cast<const uint32_t*>(&p1);
+          *reinterpret_cast<uint2*>(a.out + (static_cast<long long>(m->run_b[q]) * a.H + m->run_h[q]) *
+                                                a.d + m->run_d0[q] + 4 * x) = pk;
         }
         __syncthreads();
       }
@@ -930,30 +938,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           failed = true;
           break;
         }
-        // every segment's result is normalised (O / l) and written as bf16: a sequence held
-        // whole by this CTA straight to out; a split one to its partial slot CTA + sequence,
-        // with (m, l) beside it for the merge
+        // a sequence held whole by this CTA is normalised and written out here; a split
+        // one leaves its partial (O, m, l) in slot CTA + sequence for the merge
         const bool whole = sg.u0 == 0 && sg.u1 == seq_units(a, sg.b);
-        // the CTA's last segment: Q and the ring are idle, so the result is staged there and
-        // leaves by 1-D bulk copies instead of per-thread scalar stores
+        // the CTA's last segment: Q and the ring are idle, so the result is staged there
+        // and written with one bulk copy instead of per-thread scalar stores
         const bool staged = g == nseg - 1 && !m->more;
         const long long slot = static_cast<long long>(blockIdx.x) + sg.b;
         if (t128 < a.H) {
           const int h = t128;
           const float l = m->red[0][h] + m->red[1][h] + m->red[2][h] + m->red[3][h];
-          m->alpha[h] = 1.f / l;
-          if (!whole) {
+          if (whole) {
+            m->alpha[h] = 1.f / l;
+          } else {
             a.part_ml[(slot * a.H + h) * 2 + 0] = m_run;
             a.part_ml[(slot * a.H + h) * 2 + 1] = l;
           }
         }
-        named_bar_sync(1, 128);
-        uint16_t* dst = whole ? a.out + static_cast<long long>(sg.b) * a.H * a.d
-                              : a.part_o + slot * a.H * a.d;
-        // staged: each 128-dim block is laid out [head][128] in its own region; right after
-        // a block is complete, one thread per head stores that head's 256-byte row,
-        // overlapping the staging of the next block
-        const uint32_t blk_bytes = static_cast<uint32_t>(a.H) * 256u;
+        if (whole) named_bar_sync(1, 128);
+        float* po = a.part_o + slot * a.H * a.d;
+        uint16_t* fo = a.out + static_cast<long long>(sg.b) * a.H * a.d;
+        // staged: each 128-dim block is laid out [head][128] in its own region of the idle
+        // ring / Q buffers; right after a block is complete, one thread per head stores
+        // that head's row with a 1-D bulk copy, overlapping the staging of the next block
+        const int esz = whole ? 2 : 4;
+        const uint32_t blk_bytes = static_cast<uint32_t>(a.H) * 128u * esz;
         bool issued = false;
 #pragma unroll 1
         for (int db = 0; db < NDB; ++db) {
@@ -962,27 +971,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_wait_ld();
           const int col = db * 128 + row;       // this thread's head-dimension index
           if (staged) {
-            const uint32_t base = smem_u32(smem) + db * blk_bytes + row * 2;
+            const uint32_t base = smem_u32(smem) + db * blk_bytes + row * esz;
+            if (whole) {
 #pragma unroll
-            for (int h = 0; h < HP; ++h)
-              if (h < a.H) {
-                const __nv_bfloat16 v = __float2bfloat16_rn(ob[h] * m->alpha[h]);
-                st_shared_u16(base + h * 256u, *reinterpret_cast<const uint16_t*>(&v));
-              }
+              for (int h = 0; h < HP; ++h)
+                if (h < a.H) {
+                  const __nv_bfloat16 v = __float2bfloat16_rn(ob[h] * m->alpha[h]);
+                  st_shared_u16(base + h * 256u, *reinterpret_cast<const uint16_t*>(&v));
+                }
+            } else {
+#pragma unroll
+              for (int h = 0; h < HP; ++h)
+                if (h < a.H) st_shared_f32(base + h * 512u, ob[h]);
+            }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (t128 < a.H) {
-              bulk_store(dst + static_cast<long long>(t128) * a.d + db * 128,
-                         smem + db * blk_bytes + t128 * 256, 256u);
+              const uint8_t* src = smem + db * blk_bytes + t128 * 128 * esz;
+              if (whole)
+                bulk_store(fo + static_cast<long long>(t128) * a.d + db * 128, src, 256u);
+              else
+                bulk_store(po + static_cast<long long>(t128) * a.d + db * 128, src, 512u);
               issued = true;
             }
-          } else {
+          } else if (whole) {
 #pragma unroll
             for (int h = 0; h < HP; ++h)
               if (h < a.H) {
                 const __nv_bfloat16 v = __float2bfloat16_rn(ob[h] * m->alpha[h]);
-                dst[static_cast<long long>(h) * a.d + col] = *reinterpret_cast<const uint16_t*>(&v);
+                fo[static_cast<long long>(h) * a.d + col] = *reinterpret_cast<const uint16_t*>(&v);
               }
+          } else {
+#pragma unroll
+            for (int h = 0; h < HP; ++h)
+              if (h < a.H) po[static_cast<long long>(h) * a.d + col] = ob[h];
           }
         }
         if (issued) {
@@ -1040,14 +1062,12 @@ namespace {
 
 using lsa::attn::Args;
 
-// Workspace: bf16 normalised partial O [G+B][H][d], fp32 (m, l) [G+B][H][2], then the
-// two grid-barrier counters on their own 256-byte line.
-size_t attn_ws_body(int B, int H, int d, int n_sm) {
-  const size_t slots = static_cast<size_t>(n_sm) + static_cast<size_t>(B);
-  return slots * static_cast<size_t>(H) * (static_cast<size_t>(d) * 2 + 2 * sizeof(float));
-}
+// Workspace: fp32 partial O [G+B][H][d], partial (m, l) [G+B][H][2], then the two
+// grid-barrier counters on their own 256-byte line.
 size_t attn_ws_bytes(int B, int H, int d, int n_sm) {
-  return (attn_ws_body(B, H, d, n_sm) + 255) / 256 * 256 + 256;
+  const size_t slots = static_cast<size_t>(n_sm) + static_cast<size_t>(B);
+  const size_t body = slots * static_cast<size_t>(H) * (static_cast<size_t>(d) + 2) * sizeof(float);
+  return (body + 255) / 256 * 256 + 256;
 }
 
 template <int HP, int NDC>
@@ -1141,9 +1161,9 @@ lsa_status decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pa
   a.block_table = block_table;
   a.n_entries = n_entries;
   a.tail_len = tail_len;
-  a.part_o = static_cast<uint16_t*>(ws);
-  a.part_ml = reinterpret_cast<float*>(a.part_o + (static_cast<size_t>(G) + B) * H * d);
-  const size_t body = attn_ws_body(B, H, d, G);
+  a.part_o = static_cast<float*>(ws);
+  a.part_ml = a.part_o + (static_cast<size_t>(G) + B) * H * d;
+  const size_t body = (static_cast<size_t>(G) + B) * H * (static_cast<size_t>(d) + 2) * sizeof(float);
   a.sync = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + (body + 255) / 256 * 256);
   a.out = out;
   a.pool = const_cast<uint16_t*>(hbm_pool);
