@@ -13,7 +13,8 @@ Under torchrun every rank runs its own replica of the workload (the path has no
 exchange step at B=1), timed on the device, max over ranks.
 
 The timed region replays one CUDA graph per step (captured from the library's public
-C-ABI calls, with external timing events between the calls); `e2e` repeats the
+C-ABI calls, with external timing events after the pass set-up, the indexer, the gather
+and the last decode step); `e2e` repeats the
 measurement through lsa_step from Python with host buffers copied in and out every
 decode step.
 """
@@ -207,8 +208,8 @@ def run_pass(dec, inp, out, evs=None):
         evs[2].record()
     for s in range(inp.q.shape[0]):
         dec.decode_step(s, inp.q[s], inp.k[s], inp.v[s], out[s])
-        if evs is not None:
-            evs[3 + s].record()
+    if evs is not None:
+        evs[3].record()
 
 
 def capture(dec, inp, out, n_steps):
@@ -216,8 +217,9 @@ def capture(dec, inp, out, n_steps):
     graphs, events = [], []
     stream = torch.cuda.Stream()
     for _ in range(n_steps):
-        evs = [torch.cuda.Event(enable_timing=True, external=True)
-               for _ in range(3 + inp.q.shape[0])]
+        # four events per pass: an event node between two decode steps would cost a few
+        # microseconds of its own, so the decode steps are timed as one run of launches
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
             run_pass(dec, inp, out, evs)
@@ -227,9 +229,10 @@ def capture(dec, inp, out, n_steps):
 
 
 def event_breakdown(evs, tau):
+    """(indexer ms, gather ms, mean ms per decode-step launch) of one replayed pass."""
     idx = evs[0].elapsed_time(evs[1])
     gth = evs[1].elapsed_time(evs[2])
-    step = [evs[2 + s].elapsed_time(evs[3 + s]) for s in range(tau)]
+    step = evs[2].elapsed_time(evs[3]) / tau
     return idx, gth, step
 
 
@@ -518,7 +521,7 @@ def run_lsa(args, rank, world, local):
     idx_ms, gth_ms, attn_ms = [], [], []
     for i in range(n_graphs):
         a, g, at = event_breakdown(events[i], cfg.tau)
-        idx_ms.append(a); gth_ms.append(g); attn_ms += at
+        idx_ms.append(a); gth_ms.append(g); attn_ms.append(at)
     hbm, peak_src = peaks()
     attn_bytes = sum(attn_bytes_per_step(cfg, n_sel, s) for s in range(cfg.tau)) / cfg.tau
     attn_avg_ms = statistics.mean(attn_ms)

@@ -633,12 +633,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tensormap(&map_kv);
     prefetch_tensormap(&map_q);
   }
-  long long U = 0;
-  if (warp == 0) U = warp_total_units(a, lane);
   if (warp == 1) {
     tmem_alloc(&m->tmem_base, LY::TMEM_COLS);
     tmem_relinquish();
   }
+  // Launched as a programmatic dependent: everything above overlaps the previous
+  // kernel's tail; nothing a preceding kernel may write is read before this point.
+  grid_dependency_wait();
+  grid_dependents_launch();
+  long long U = 0;
+  if (warp == 0) U = warp_total_units(a, lane);
   // grid-wide split of the batch's units
   const long long G = gridDim.x;
   long long us = 0, ue = 0;
@@ -1091,10 +1095,20 @@ lsa_status launch_attn(const CUtensorMap& mkv, const CUtensorMap& mq, const Args
   cfg.blockDim = dim3(lsa::attn::NTHREADS);
   cfg.dynamicSmemBytes = LY::SMEM;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  // Programmatic stream serialisation lets this launch's CTAs set up while the previous
+  // kernel in the stream drains; the kernel waits for it before touching any data.
+  static bool pdl_ok = true;
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
+  cfg.numAttrs = pdl_ok ? 2 : 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mkv, mq, a) == cudaSuccess) return LSA_OK;
+  cudaGetLastError();
+  if (!pdl_ok) return LSA_ERR_CUDA;
+  pdl_ok = false;  // this driver refuses the combination: plain cooperative launches
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, mkv, mq, a) != cudaSuccess) {
     cudaGetLastError();
