@@ -83,8 +83,12 @@ int32_t lsa_version(void);
  *                                     untouched)
  *   layer_mask nullable device u32 [L+1][B][ceil(max_cand/32)] out: bit c%32 of word
  *             c/32 = (z_l > 0) for l < L, and the OR for l = L
- *   ws        device workspace of lsa_index_workspace_size(B, L, d_i, max_cand) bytes
- * Supported: 1 <= L <= 4, d_i == 128, D % 256 == 0, B >= 1, cap >= 0.
+ *   ws        device workspace of lsa_index_workspace_size(B, L, d_i, max_cand) bytes,
+ *             16-byte aligned, zero-filled before the first call (every call leaves its
+ *             grid-barrier counters zero again)
+ * Supported: 1 <= L <= 4, d_i == 128, D % 256 == 0, B >= 1, cap >= 0. One cooperative
+ * launch (one CTA per SM, all resident) with two grid-wide barriers: projection, then
+ * scoring, then compaction.
  */
 lsa_status lsa_index(const uint16_t* h, const uint16_t* w_q, const float* bias,
                      const uint16_t* k_idx, const int64_t* kidx_off, const int32_t* n_cand,
@@ -150,7 +154,9 @@ lsa_status lsa_gather(const uint16_t* host_pool, int64_t host_blocks,
  * Supported: d in {128, 256, 384, 512}, 1 <= H <= 64, scale > 0, n_pages <= 2^23,
  *            q, hbm_pool, ws and out 16-byte aligned. The launch is cooperative (one
  *            CTA per SM, all resident): the partial results are merged inside the same
- *            kernel behind a grid-wide barrier whose counters live in ws.
+ *            kernel behind a grid-wide barrier whose counters live in the first 256
+ *            bytes of ws: they must be zero before the first call, and every call
+ *            leaves them zero, so one workspace serves calls of any shape in turn.
  */
 lsa_status lsa_decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pages,
                            const int32_t* block_table, int32_t bt_stride,

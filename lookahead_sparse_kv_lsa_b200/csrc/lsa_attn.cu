@@ -597,7 +597,8 @@ struct Layout {
 template <int HP, int NDC>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_splitk_kernel(const __grid_constant__ CUtensorMap map_kv,
-                       const __grid_constant__ CUtensorMap map_q, const Args a) {
+                       const __grid_constant__ CUtensorMap map_q,
+                       const __grid_constant__ Args a) {
   using LY = Layout<HP, NDC>;
   constexpr int NDB = LY::NDB;
   extern __shared__ uint8_t smem_raw[];
@@ -1066,8 +1067,8 @@ namespace {
 
 using lsa::attn::Args;
 
-// Workspace: fp32 partial O [G+B][H][d], partial (m, l) [G+B][H][2], then the two
-// grid-barrier counters on their own 256-byte line.
+// Workspace: the two grid-barrier counters on their own 256-byte line, then fp32
+// partial O [G+B][H][d] and partial (m, l) [G+B][H][2].
 size_t attn_ws_bytes(int B, int H, int d, int n_sm) {
   const size_t slots = static_cast<size_t>(n_sm) + static_cast<size_t>(B);
   const size_t body = slots * static_cast<size_t>(H) * (static_cast<size_t>(d) + 2) * sizeof(float);
@@ -1175,10 +1176,11 @@ lsa_status decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pa
   a.block_table = block_table;
   a.n_entries = n_entries;
   a.tail_len = tail_len;
-  a.part_o = static_cast<float*>(ws);
+  // the barrier counters sit at a fixed place (the first 256 bytes) whatever the shape,
+  // so one array can serve calls of different shapes in turn
+  a.sync = static_cast<unsigned int*>(ws);
+  a.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 256);
   a.part_ml = a.part_o + (static_cast<size_t>(G) + B) * H * d;
-  const size_t body = (static_cast<size_t>(G) + B) * H * (static_cast<size_t>(d) + 2) * sizeof(float);
-  a.sync = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + (body + 255) / 256 * 256);
   a.out = out;
   a.pool = const_cast<uint16_t*>(hbm_pool);
   if (append) {

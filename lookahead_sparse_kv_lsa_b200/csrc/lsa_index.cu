@@ -6,14 +6,23 @@
 // small query projection per layer against frozen compressed block keys), section 4
 // (independent indexers at three layers, OR-ed).
 //
-// Two kernels:
-//  1. project: q[l][b][:] = W_q[l] . h[l][b] in fp32 (one warp per output row, bf16
-//     operands read with 16-byte loads, fixed-order warp reduction);
-//  2. score: 16 lanes per candidate row (16 bytes each, so a warp reads two 256-byte
-//     K_idx rows per load, coalesced), z_l = q_l . k / sqrt(d_i) + bias, keep bit
-//     z_l > 0 (equal to sigmoid(z_l) > 0.5), OR over the layers, packed with warp
-//     ballots into 32-bit words. The last CTA of each sequence (atomic ticket, no
-//     waiting) turns the words into the ascending id list with a block prefix sum.
+// One cooperative launch, one CTA per SM, three phases split by two grid barriers:
+//
+//  A. Each CTA starts 1-D bulk copies of its share of K_idx into shared memory (it does
+//     not depend on q), then computes its share of the W_q rows: q[l][b][j] = W_q[l][j] .
+//     h[l][b] in fp32, each dot cut into four fixed parts summed in a fixed order.
+//  B. Scoring. The candidate rows of every sequence are grouped in 32-row "words"; all
+//     words of the batch, in sequence order, are divided evenly over the CTAs. A warp
+//     scores one word from shared memory, 8 lanes per row (16 bytes of the row each, so
+//     the 4 rows a load instruction covers fall in disjoint banks):
+//     z_l = q_l . k / sqrt(d_i) + bias, keep bit z_l > 0 (equal to sigmoid(z_l) > 0.5),
+//     OR over the layers, collected into the word with warp ballots.
+//  C. Compaction. Each CTA ranks the kept bits of its words (popcounts of the earlier
+//     words of the same sequence, a block scan over its own) and writes the ascending id
+//     list; the CTA holding a sequence's last word writes its count.
+//
+// Grid barriers use an arrival counter in the workspace with a bounded wait; the last
+// CTA to leave resets the counters, so the workspace is left as it was found (zero).
 #include "lsa_common.cuh"
 
 namespace lsa {
@@ -21,15 +30,61 @@ namespace idx {
 
 constexpr int D_I = 128;
 constexpr int MAX_L = 4;
-constexpr int PROJ_WARPS = 4;        // output rows per projection CTA
-constexpr int PROJ_BCHUNK = 8;       // sequences accumulated at once per warp
-constexpr int SCORE_WARPS = 8;
-constexpr int ROWS_PER_CTA = SCORE_WARPS * 32;
+constexpr int NTHREADS = 256;
+constexpr int NWARPS = NTHREADS / 32;
+constexpr int WORD_ROWS = 32;                       // candidate rows per keep word
+constexpr int ROW_BYTES = D_I * 2;                  // one K_idx row, bf16
+constexpr int WORD_BYTES = WORD_ROWS * ROW_BYTES;   // 8 KB
+constexpr int CHUNK_WORDS = 20;                     // K_idx words resident at once (160 KB)
+constexpr int NPART = 4;                            // projection: parts per dot product
+constexpr int RMAX = 4;                             // projection: W_q rows per round
+constexpr int BCH = 32;                             // projection: sequences per round
+constexpr int MAX_GRID = 1024;
 
-struct Ws {
-  float* q;            // [L][B][D_I]
-  uint32_t* words;     // [B][n_words]   OR keep bits
-  int32_t* ticket;     // [B]
+struct Args {
+  const uint16_t* h;         // [L][B][D]
+  const uint16_t* w_q;       // [L][D_I][D]
+  const float* bias;         // [B]
+  const uint16_t* k_idx;     // [rows][D_I]
+  const int64_t* kidx_off;   // [B]
+  const int32_t* n_cand;     // [B]
+  float* q;                  // workspace [L][B][D_I]
+  uint32_t* words;           // workspace [B][n_words]: OR keep bits
+  unsigned int* sync;        // workspace [2]: barrier arrivals, departures
+  int32_t* sel_ids;          // [B][cap]
+  int32_t* sel_cnt;          // [B]
+  float* logits;             // nullable [L][B][max_cand]
+  uint32_t* layer_mask;      // nullable [L+1][B][mask_words]
+  int32_t* err;
+  int B, L, D, max_cand, n_words, mask_words, cap;
+  float inv_sqrt_di;
+};
+
+// Sequences met by a range of words (at most CHUNK_WORDS words, so at most as many
+// sequences): first word index, words, candidates, K_idx row of block 0, bias.
+struct SeqTab {
+  int n;
+  int b[CHUNK_WORDS];
+  long long w0[CHUNK_WORDS];
+  int nw[CHUNK_WORDS];
+  int nc[CHUNK_WORDS];
+  long long row0[CHUNK_WORDS];
+  float bias[CHUNK_WORDS];
+  int resume_b;              // walk state for the next range
+  long long resume_base;
+};
+
+struct Smem {
+  uint8_t kbuf[CHUNK_WORDS * WORD_BYTES];
+  uint64_t kbar;
+  int abort;
+  int word_seq[CHUNK_WORDS];             // table entry of each word of the chunk
+  uint32_t wbits[MAX_L][CHUNK_WORDS];    // keep bits of the chunk's words, per layer
+  alignas(16) float qs[CHUNK_WORDS][MAX_L][D_I];   // queries of the chunk's sequences
+  int red[NWARPS];
+  SeqTab tab;
+  float part[RMAX][BCH][NPART];          // projection partial sums
+  long long nw_total;
 };
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
@@ -41,68 +96,9 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   }
 }
 
-// q[l][b][j] = sum_i W_q[l][j][i] * h[l][b][i]
-__global__ void __launch_bounds__(PROJ_WARPS * 32)
-    project_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ w_q, int B, int L,
-                   int D, float* __restrict__ q) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * PROJ_WARPS + warp;  // l * D_I + j
-  if (row >= L * D_I) return;
-  const int l = row / D_I, j = row % D_I;
-  const uint4* wrow = reinterpret_cast<const uint4*>(w_q + static_cast<size_t>(row) * D);
-  const int n_it = D / 256;
-  for (int b0 = 0; b0 < B; b0 += PROJ_BCHUNK) {
-    float acc[PROJ_BCHUNK];
-#pragma unroll
-    for (int k = 0; k < PROJ_BCHUNK; ++k) acc[k] = 0.f;
-#pragma unroll 4
-    for (int it = 0; it < n_it; ++it) {
-      float wf[8];
-      unpack8(__ldg(wrow + it * 32 + lane), wf);
-#pragma unroll
-      for (int k = 0; k < PROJ_BCHUNK; ++k) {
-        const int b = b0 + k;
-        if (b < B) {
-          const uint4* hrow =
-              reinterpret_cast<const uint4*>(h + (static_cast<size_t>(l) * B + b) * D);
-          float hf[8];
-          unpack8(__ldg(hrow + it * 32 + lane), hf);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[k] = fmaf(wf[e], hf[e], acc[k]);
-        }
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < PROJ_BCHUNK; ++k) {
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int k = 0; k < PROJ_BCHUNK; ++k)
-        if (b0 + k < B) q[(static_cast<size_t>(l) * B + b0 + k) * D_I + j] = acc[k];
-    }
-  }
-}
-
-struct ScoreArgs {
-  const uint16_t* k_idx;
-  const int64_t* kidx_off;
-  const int32_t* n_cand;
-  const float* bias;
-  const float* q;          // [L][B][D_I]
-  uint32_t* words;         // [B][n_words]
-  int32_t* ticket;         // [B]
-  int32_t* sel_ids;        // [B][cap]
-  int32_t* sel_cnt;        // [B]
-  float* logits;           // nullable [L][B][max_cand]
-  uint32_t* layer_mask;    // nullable [L+1][B][n_words]
-  int32_t* err;
-  int B, L, max_cand, n_words, mask_words, cap;
-  float inv_sqrt_di;
-};
-
-__device__ __forceinline__ int clamp_cand(const ScoreArgs& a, int b, bool report) {
+// Candidates of sequence b, clamped to [0, max_cand] (out-of-range counts are reported
+// by the CTA that `report`s).
+__device__ __forceinline__ int seq_cand(const Args& a, int b, bool report) {
   int n = __ldg(a.n_cand + b);
   if (n < 0 || n > a.max_cand) {
     if (report) set_err(a.err, LSA_DEVERR_BAD_SIZE);
@@ -110,127 +106,430 @@ __device__ __forceinline__ int clamp_cand(const ScoreArgs& a, int b, bool report
   }
   return n;
 }
+__device__ __forceinline__ int seq_words(int n) { return (n + WORD_ROWS - 1) / WORD_ROWS; }
 
-// grid (ceil(max_cand / ROWS_PER_CTA), B); CTA x of sequence b scores candidates
-// [x*256, x*256+256) in 8 warps of 32 rows, 2 rows per load (16 lanes per row).
-__global__ void __launch_bounds__(SCORE_WARPS * 32) score_kernel(const ScoreArgs a) {
-  const int b = blockIdx.y;
-  const int n = clamp_cand(a, b, blockIdx.x == 0 && threadIdx.x == 0);
-  const int n_cta = max(1, (n + ROWS_PER_CTA - 1) / ROWS_PER_CTA);
-  if (static_cast<int>(blockIdx.x) >= n_cta) return;
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = lane >> 4, sub = lane & 15;
-  const int L = a.L;
-  // this lane's 8-element slice of each layer's query
-  float qv[MAX_L][8];
-#pragma unroll
-  for (int l = 0; l < MAX_L; ++l) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      qv[l][e] = l < L ? a.q[(static_cast<size_t>(l) * a.B + b) * D_I + sub * 8 + e] : 0.f;
+// Total keep words of the batch, summed by one warp (every lane gets it). The first 32
+// sequences' K_idx offsets and biases, which the plan reads next, are prefetched.
+__device__ __forceinline__ long long warp_total_words(const Args& a, int lane) {
+  if (lane < a.B) {
+    prefetch_l1(a.kidx_off + lane);
+    prefetch_l1(a.bias + lane);
   }
-  const float bias = __ldg(a.bias + b);
-  const int c_base = blockIdx.x * ROWS_PER_CTA + warp * 32;
-  const uint4* kb = reinterpret_cast<const uint4*>(a.k_idx + __ldg(a.kidx_off + b) * D_I);
+  long long s = 0;
+  for (int b = lane; b < a.B; b += 32) s += seq_words(seq_cand(a, b, false));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
 
-  // issue all 16 loads of the warp's 32 rows first (16 B per lane each)
-  uint4 kv[16];
-#pragma unroll
-  for (int it = 0; it < 16; ++it) {
-    const int c = c_base + 2 * it + half;
-    kv[it] = c < n ? __ldg(kb + static_cast<size_t>(c) * (D_I / 8) + sub) : make_uint4(0, 0, 0, 0);
-  }
-  uint32_t w_or = 0;
-  uint32_t w_l[MAX_L] = {0, 0, 0, 0};
-#pragma unroll
-  for (int it = 0; it < 16; ++it) {
-    const int c = c_base + 2 * it + half;
-    float kf[8];
-    unpack8(kv[it], kf);
-    bool any = false;
-#pragma unroll
-    for (int l = 0; l < MAX_L; ++l) {
-      if (l < L) {
-        float s = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s = fmaf(qv[l][e], kf[e], s);
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        const float z = fmaf(s, a.inv_sqrt_di, bias);
-        const bool keep = (c < n) && (z > 0.f);
-        any |= keep;
-        if (a.logits != nullptr && sub == 0 && c < n)
-          a.logits[(static_cast<size_t>(l) * a.B + b) * a.max_cand + c] = z;
-        const uint32_t bal = __ballot_sync(0xffffffffu, keep && sub == 0);
-        w_l[l] |= ((bal & 1u) << (2 * it)) | (((bal >> 16) & 1u) << (2 * it + 1));
-      }
-    }
-    const uint32_t bal = __ballot_sync(0xffffffffu, any && sub == 0);
-    w_or |= ((bal & 1u) << (2 * it)) | (((bal >> 16) & 1u) << (2 * it + 1));
-  }
-  const int word = c_base >> 5;
-  if (lane == 0 && c_base < n) {
-    a.words[static_cast<size_t>(b) * a.n_words + word] = w_or;
-    if (a.layer_mask != nullptr) {
-      for (int l = 0; l < L; ++l)
-        a.layer_mask[(static_cast<size_t>(l) * a.B + b) * a.mask_words + word] = w_l[l];
-      a.layer_mask[(static_cast<size_t>(L) * a.B + b) * a.mask_words + word] = w_or;
-    }
-  }
-
-  // ---- last CTA of this sequence compacts the id list (no CTA ever waits)
-  __shared__ int s_last;
-  __shared__ int s_warp[SCORE_WARPS];
-  __shared__ int s_carry;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int t = atomicAdd(a.ticket + b, 1);
-    s_last = (t == n_cta - 1);
-    s_carry = 0;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const int n_w = (n + 31) >> 5;
-  const uint32_t* words = a.words + static_cast<size_t>(b) * a.n_words;
-  int32_t* out = a.sel_ids + static_cast<size_t>(b) * a.cap;
-  for (int w0 = 0; w0 < n_w; w0 += SCORE_WARPS * 32) {
-    const int w = w0 + threadIdx.x;
-    const uint32_t bits = w < n_w ? __ldcg(words + w) : 0u;
-    const int cnt = __popc(bits);
-    int incl = cnt;
+// Warp 0: fill t with the sequences that own words of [w_lo, w_hi), walking forward
+// from the saved state (sequence resume_b, whose first word is resume_base).
+__device__ __forceinline__ void plan_words(const Args& a, long long w_lo, long long w_hi, SeqTab* t,
+                                          int lane) {
+  int found = 0;
+  long long base = t->resume_base;
+  int last_b = t->resume_b;
+  long long last_base = t->resume_base;
+  for (int b0 = t->resume_b; b0 < a.B && base < w_hi; b0 += 32) {
+    const int b = b0 + lane;
+    const int n = b < a.B ? seq_cand(a, b, false) : 0;
+    const long long row0 = b < a.B ? __ldg(a.kidx_off + b) : 0;   // loaded with n
+    const float bias = b < a.B ? __ldg(a.bias + b) : 0.f;
+    const int nw = seq_words(n);
+    long long incl = nw;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
+      const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    int before = s_carry;
-    for (int k = 0; k < warp; ++k) before += s_warp[k];
-    int pos = before + incl - cnt;
+    const long long p = base + incl - nw;     // first word of sequence b
+    const bool hit = nw > 0 && p < w_hi && p + nw > w_lo;
+    const unsigned mask = __ballot_sync(0xffffffffu, hit);
+    if (hit) {
+      const int i = found + __popc(mask & ((1u << lane) - 1u));
+      if (i < CHUNK_WORDS) {
+        t->b[i] = b;
+        t->w0[i] = p;
+        t->nw[i] = nw;
+        t->nc[i] = n;
+        t->row0[i] = row0;
+        t->bias[i] = bias;
+      }
+    }
+    if (mask != 0) {
+      const int hi_lane = 31 - __clz(mask);
+      last_b = __shfl_sync(0xffffffffu, b, hi_lane);
+      last_base = __shfl_sync(0xffffffffu, p, hi_lane);
+    }
+    found += __popc(mask);
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) {
+    t->n = found < CHUNK_WORDS ? found : CHUNK_WORDS;
+    t->resume_b = last_b;          // the last sequence met may continue into the next range
+    t->resume_base = last_base;
+  }
+}
+
+// Grid-wide barrier number k (1, 2, ...): every CTA arrives; the wait is bounded and,
+// once the CTA has given up (abort), it still arrives but no longer waits.
+__device__ __forceinline__ void grid_sync(const Args& a, Smem* s, unsigned int k) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(a.sync, 1u);
+    const unsigned int target = k * gridDim.x;
+    if (!s->abort) {
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_gpu(a.sync) < target) {
+        __nanosleep(32);
+        if (globaltimer_ns() - t0 > LSA_WAIT_LIMIT_NS) {
+          set_err(a.err, LSA_DEVERR_TIMEOUT);
+          s->abort = 1;
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+}
+
+// Warp 0: plan the chunk [cw0, cw1) of keep words and start the bulk copies of their
+// K_idx rows into s->kbuf (one copy per word; a sequence's last word may be partial).
+__device__ __forceinline__ void issue_chunk(const Args& a, Smem* s, long long cw0, long long cw1,
+                                            int lane) {
+  plan_words(a, cw0, cw1, &s->tab, lane);
+  __syncwarp();
+  const int nwc = static_cast<int>(cw1 - cw0);
+  uint32_t bytes = 0;
+  const uint16_t* src = nullptr;
+  if (lane < nwc) {
+    const long long w = cw0 + lane;
+    int i = 0;
+    while (i + 1 < s->tab.n && s->tab.w0[i + 1] <= w) ++i;
+    const int wi = static_cast<int>(w - s->tab.w0[i]);
+    const int rows = min(WORD_ROWS, s->tab.nc[i] - WORD_ROWS * wi);
+    bytes = static_cast<uint32_t>(rows) * ROW_BYTES;
+    src = a.k_idx + (s->tab.row0[i] + static_cast<long long>(WORD_ROWS) * wi) * D_I;
+    s->word_seq[lane] = i;
+  }
+  uint32_t total = bytes;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+  if (lane == 0) {
+    fence_proxy_async_smem();          // earlier generic reads of kbuf before the refill
+    mbar_arrive_expect_tx(&s->kbar, total);
+  }
+  __syncwarp();
+  if (lane < nwc) bulk_load(s->kbuf + lane * WORD_BYTES, src, bytes, &s->kbar);
+}
+
+// All threads: stage the queries of the chunk's sequences in shared memory and clear
+// the chunk's keep bits (one round trip to L2 for the whole CTA).
+__device__ __forceinline__ void stage_queries(const Args& a, Smem* s) {
+  const int per_seq = a.L * (D_I / 4);                  // float4s per sequence
+  const int total = s->tab.n * per_seq;
+  for (int i = threadIdx.x; i < total; i += NTHREADS) {
+    const int e = i / per_seq, r = i - e * per_seq;
+    const int l = r / (D_I / 4), c4 = r - l * (D_I / 4);
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                                a.q + (static_cast<long long>(l) * a.B + s->tab.b[e]) * D_I) + c4);
+    *reinterpret_cast<float4*>(&s->qs[e][l][4 * c4]) = v;
+  }
+  for (int i = threadIdx.x; i < MAX_L * CHUNK_WORDS; i += NTHREADS) (&s->wbits[0][0])[i] = 0u;
+}
+
+// Warp: rows 4*st .. 4*st+3 of keep word k of the current chunk, 8 lanes per row (lane
+// sub reads 16-byte pieces sub and sub+8 of its row). The 4 keep bits of each layer go
+// into the word's bits in shared memory.
+__device__ __forceinline__ void score_rows(const Args& a, Smem* s, int k, int st, long long cw0,
+                                           int lane) {
+  const int i = s->word_seq[k];
+  const int wi = static_cast<int>(cw0 + k - s->tab.w0[i]);
+  const int n = s->tab.nc[i];
+  const float bias = s->tab.bias[i];
+  const int sub = lane & 7;
+  const int rl = 4 * st + (lane >> 3);
+  const int c = WORD_ROWS * wi + rl;
+  const bool valid = c < n;
+  const uint8_t* rp = s->kbuf + k * WORD_BYTES + rl * ROW_BYTES + 16 * sub;
+  float k0[8], k1[8];
+  unpack8(*reinterpret_cast<const uint4*>(rp), k0);
+  unpack8(*reinterpret_cast<const uint4*>(rp + 128), k1);
+  float z[MAX_L];
+#pragma unroll
+  for (int l = 0; l < MAX_L; ++l) {
+    if (l < a.L) {
+      const float4* q0 = reinterpret_cast<const float4*>(&s->qs[i][l][8 * sub]);
+      const float4* q1 = reinterpret_cast<const float4*>(&s->qs[i][l][64 + 8 * sub]);
+      const float4 qa = q0[0], qb = q0[1], qc = q1[0], qd = q1[1];
+      // two independent chains, joined in a fixed order
+      float u = qa.x * k0[0], v = qc.x * k1[0];
+      u = fmaf(qa.y, k0[1], u); v = fmaf(qc.y, k1[1], v);
+      u = fmaf(qa.z, k0[2], u); v = fmaf(qc.z, k1[2], v);
+      u = fmaf(qa.w, k0[3], u); v = fmaf(qc.w, k1[3], v);
+      u = fmaf(qb.x, k0[4], u); v = fmaf(qd.x, k1[4], v);
+      u = fmaf(qb.y, k0[5], u); v = fmaf(qd.y, k1[5], v);
+      u = fmaf(qb.z, k0[6], u); v = fmaf(qd.z, k1[6], v);
+      u = fmaf(qb.w, k0[7], u); v = fmaf(qd.w, k1[7], v);
+      z[l] = u + v;
+    }
+  }
+#pragma unroll
+  for (int o = 4; o >= 1; o >>= 1) {
+#pragma unroll
+    for (int l = 0; l < MAX_L; ++l)
+      if (l < a.L) z[l] += __shfl_xor_sync(0xffffffffu, z[l], o);
+  }
+  const int b = s->tab.b[i];
+#pragma unroll
+  for (int l = 0; l < MAX_L; ++l) {
+    if (l < a.L) {
+      const float zz = fmaf(z[l], a.inv_sqrt_di, bias);
+      const bool keep = valid && zz > 0.f;
+      if (a.logits != nullptr && sub == 0 && valid)
+        a.logits[(static_cast<long long>(l) * a.B + b) * a.max_cand + c] = zz;
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep && sub == 0);
+      const uint32_t nib = (bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u);
+      if (lane == 0 && nib != 0u) atomicOr(&s->wbits[l][k], nib << (4 * st));
+    }
+  }
+}
+
+// Threads: write the chunk's keep words (OR over the layers, and the per-layer masks).
+__device__ __forceinline__ void store_words(const Args& a, Smem* s, int nwc, long long cw0) {
+  for (int k = threadIdx.x; k < nwc; k += NTHREADS) {
+    const int i = s->word_seq[k];
+    const int b = s->tab.b[i];
+    const int wi = static_cast<int>(cw0 + k - s->tab.w0[i]);
+    uint32_t wor = 0;
+#pragma unroll
+    for (int l = 0; l < MAX_L; ++l)
+      if (l < a.L) wor |= s->wbits[l][k];
+    a.words[static_cast<long long>(b) * a.n_words + wi] = wor;
+    if (a.layer_mask != nullptr) {
+#pragma unroll
+      for (int l = 0; l < MAX_L; ++l)
+        if (l < a.L)
+          a.layer_mask[(static_cast<long long>(l) * a.B + b) * a.mask_words + wi] = s->wbits[l][k];
+      a.layer_mask[(static_cast<long long>(a.L) * a.B + b) * a.mask_words + wi] = wor;
+    }
+  }
+}
+
+// Warps 1.. (PROJ_THREADS threads, named barrier 1): q rows [r_lo, r_hi) of the stacked
+// W_q (row = l * D_I + j) for every sequence. Each dot product is cut into NPART parts of
+// whole 8-element groups; a warp sums one part (lane-strided, then a butterfly), and the
+// parts are added in order.
+constexpr int PROJ_THREADS = NTHREADS - 32;
+constexpr int PROJ_WARPS = PROJ_THREADS / 32;
+__device__ __forceinline__ void project_rows(const Args& a, Smem* s, int r_lo, int r_hi) {
+  const int tid = threadIdx.x - 32, warp = tid >> 5, lane = tid & 31;
+  const int g8 = a.D / 8;
+  for (int rg = r_lo; rg < r_hi; rg += RMAX) {
+    const int nr = min(RMAX, r_hi - rg);
+    for (int b0 = 0; b0 < a.B; b0 += BCH) {
+      const int nb = min(BCH, a.B - b0);
+      const int tasks = nr * nb * NPART;
+      for (int t = warp; t < tasks; t += PROJ_WARPS) {
+        const int p = t % NPART;
+        const int rb = t / NPART;
+        const int bl = rb % nb, r = rb / nb;
+        const int row = rg + r;
+        const int l = row / D_I;
+        const uint4* wrow = reinterpret_cast<const uint4*>(a.w_q + static_cast<long long>(row) * a.D);
+        const uint4* hrow =
+            reinterpret_cast<const uint4*>(a.h + (static_cast<long long>(l) * a.B + b0 + bl) * a.D);
+        const int g_lo = (p * g8) / NPART, g_hi = ((p + 1) * g8) / NPART;
+        float acc = 0.f;
+#pragma unroll 4
+        for (int g = g_lo + lane; g < g_hi; g += 32) {
+          float wf[8], hf[8];
+          unpack8(__ldg(wrow + g), wf);
+          unpack8(__ldg(hrow + g), hf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc = fmaf(wf[e], hf[e], acc);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) s->part[r][bl][p] = acc;
+      }
+      named_bar_sync(1, PROJ_THREADS);
+      for (int i = tid; i < nr * nb; i += PROJ_THREADS) {
+        const int r = i / nb, bl = i % nb;
+        float sum = 0.f;
+#pragma unroll
+        for (int p = 0; p < NPART; ++p) sum += s->part[r][bl][p];
+        const int row = rg + r;
+        const int l = row / D_I, j = row % D_I;
+        a.q[(static_cast<long long>(l) * a.B + b0 + bl) * D_I + j] = sum;
+      }
+      named_bar_sync(1, PROJ_THREADS);
+    }
+  }
+}
+
+// Warp 0: ids of the keep words [dw0, dw1) (at most CHUNK_WORDS, planned in s->tab).
+// `carry` = kept blocks of the chunk's first sequence in words before dw0; returns the
+// same for the next chunk.
+__device__ __forceinline__ int compact_chunk(const Args& a, Smem* s, long long dw0, long long dw1,
+                                             int carry, int lane) {
+  const int nwc = static_cast<int>(dw1 - dw0);
+  int i = 0, b = 0, wi = 0, ts = 0;
+  uint32_t bits = 0;
+  if (lane < nwc) {
+    const long long w = dw0 + lane;
+    while (i + 1 < s->tab.n && s->tab.w0[i + 1] <= w) ++i;
+    b = s->tab.b[i];
+    wi = static_cast<int>(w - s->tab.w0[i]);
+    ts = s->tab.w0[i] > dw0 ? static_cast<int>(s->tab.w0[i] - dw0) : 0;  // lane of its 1st word
+    bits = __ldcg(a.words + static_cast<long long>(b) * a.n_words + wi);
+  }
+  const int cnt = __popc(bits);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int excl = incl - cnt;
+  const int ex_ts = __shfl_sync(0xffffffffu, excl, ts);
+  const int base = (lane < nwc && s->tab.w0[i] < dw0) ? carry : 0;
+  if (lane < nwc) {
+    int pos = base + excl - ex_ts;
+    int32_t* out = a.sel_ids + static_cast<long long>(b) * a.cap;
     uint32_t rem = bits;
     while (rem) {
       const int bit = __ffs(rem) - 1;
       rem &= rem - 1;
-      if (pos < a.cap) out[pos] = w * 32 + bit;
+      if (pos < a.cap) out[pos] = WORD_ROWS * wi + bit;
       ++pos;
     }
+    if (wi == s->tab.nw[i] - 1) {        // the sequence's last word: its count
+      if (pos > a.cap) set_err(a.err, LSA_DEVERR_SEL_CAPACITY);
+      a.sel_cnt[b] = pos < a.cap ? pos : a.cap;
+    }
+  }
+  // the next chunk's carry: the last sequence's kept blocks so far
+  const int last = nwc - 1;
+  const int ts_last = __shfl_sync(0xffffffffu, ts, last);
+  const int base_last = __shfl_sync(0xffffffffu, base, last);
+  const int incl_last = __shfl_sync(0xffffffffu, incl, last);
+  const int ex_last = __shfl_sync(0xffffffffu, excl, ts_last);
+  return base_last + incl_last - ex_last;
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem* s = reinterpret_cast<Smem*>(smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long G = gridDim.x;
+  const int cta = blockIdx.x;
+
+  if (tid == 0) {
+    mbar_init(&s->kbar, 1);
+    s->abort = 0;
+    s->tab.resume_b = 0;
+    s->tab.resume_base = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // ---- phase A. Warp 0: this CTA's keep words [W0, W1), whose first chunk of K_idx
+  // loads goes out at once; warps 1..: this CTA's rows of q.
+  if (warp == 0) {
+    const long long NW = warp_total_words(a, lane);
+    const long long W0 = (cta * NW) / G, W1 = ((cta + 1) * NW) / G;
+    if (W1 > W0) issue_chunk(a, s, W0, W1 < W0 + CHUNK_WORDS ? W1 : W0 + CHUNK_WORDS, lane);
+    if (lane == 0) s->nw_total = NW;
+  } else {
+    const int RQ = a.L * D_I;
+    project_rows(a, s, static_cast<int>((cta * RQ) / G), static_cast<int>(((cta + 1) * RQ) / G));
+  }
+  grid_sync(a, s, 1);
+  const long long NW = s->nw_total;
+  const long long W0 = (cta * NW) / G, W1 = ((cta + 1) * NW) / G;
+
+  // ---- phase B: keep words
+  uint32_t parity = 0;
+  for (long long cw0 = W0; cw0 < W1; cw0 += CHUNK_WORDS) {
+    const long long cw1 = W1 < cw0 + CHUNK_WORDS ? W1 : cw0 + CHUNK_WORDS;
+    if (cw0 != W0) {
+      __syncthreads();                          // every warp is done with kbuf
+      if (warp == 0) issue_chunk(a, s, cw0, cw1, lane);
+      __syncthreads();
+    }
+    // always wait for the copies in flight, even after an abort (bounded)
+    const bool landed = mbar_wait(&s->kbar, parity, nullptr);
+    parity ^= 1u;
+    if (!landed && tid == 0) {
+      set_err(a.err, LSA_DEVERR_TIMEOUT);
+      s->abort = 1;
+    }
+    if (!s->abort) stage_queries(a, s);
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int tot = 0;
-      for (int k = 0; k < SCORE_WARPS; ++k) tot += s_warp[k];
-      s_carry += tot;
+    if (s->abort) break;
+    // tasks (word, 4-row step) round-robin over the warps: a warp's tasks are independent
+    const int nwc = static_cast<int>(cw1 - cw0);
+    for (int t = warp; t < nwc * (WORD_ROWS / 4); t += NWARPS)
+      score_rows(a, s, t >> 3, t & 7, cw0, lane);
+    __syncthreads();
+    store_words(a, s, nwc, cw0);
+  }
+  grid_sync(a, s, 2);
+
+  // ---- phase C: ordered ids
+  if (!s->abort && W1 > W0) {            // the same branch in every thread of the CTA
+    if (warp == 0) {
+      s->tab.resume_b = 0;
+      s->tab.resume_base = 0;
+      plan_words(a, W0, W1 < W0 + CHUNK_WORDS ? W1 : W0 + CHUNK_WORDS, &s->tab, lane);
     }
     __syncthreads();
+    // kept blocks of the first sequence in its words before W0, summed by the CTA
+    int part = 0;
+    const long long first = s->tab.w0[0];
+    if (first < W0) {
+      const long long wrow = static_cast<long long>(s->tab.b[0]) * a.n_words;
+      const int skip = static_cast<int>(W0 - first);
+      for (int w = tid; w < skip; w += NTHREADS) part += __popc(__ldcg(a.words + wrow + w));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) s->red[warp] = part;
+    __syncthreads();
+    if (warp == 0) {
+      int carry = 0;
+#pragma unroll
+      for (int w = 0; w < NWARPS; ++w) carry += s->red[w];
+      for (long long dw0 = W0; dw0 < W1; dw0 += CHUNK_WORDS) {
+        const long long dw1 = W1 < dw0 + CHUNK_WORDS ? W1 : dw0 + CHUNK_WORDS;
+        if (dw0 != W0) {
+          plan_words(a, dw0, dw1, &s->tab, lane);
+          __syncwarp();
+        }
+        carry = compact_chunk(a, s, dw0, dw1, carry, lane);
+        __syncwarp();
+      }
+    }
   }
-  if (threadIdx.x == 0) {
-    const int total = s_carry;
-    if (total > a.cap) set_err(a.err, LSA_DEVERR_SEL_CAPACITY);
-    a.sel_cnt[b] = min(total, a.cap);
-    a.ticket[b] = 0;  // ready for the next pass
+
+  // sequences without candidates get a zero count; bad counts are reported once
+  for (long long b = static_cast<long long>(cta) * NTHREADS + tid; b < a.B; b += G * NTHREADS) {
+    if (seq_cand(a, static_cast<int>(b), true) == 0) a.sel_cnt[b] = 0;
+  }
+
+  // ---- departure: the last CTA out resets the barrier counters
+  __syncthreads();
+  if (tid == 0) {
+    if (atomicAdd(a.sync + 1, 1u) == static_cast<unsigned int>(G) - 1u) {
+      atomicExch(a.sync, 0u);
+      atomicExch(a.sync + 1, 0u);
+    }
   }
 }
 
@@ -241,8 +540,10 @@ __global__ void __launch_bounds__(SCORE_WARPS * 32) score_kernel(const ScoreArgs
 namespace {
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Workspace: q fp32 [L][B][d_i], keep words u32 [B][n_words], then the two grid-barrier
+// counters on their own 256-byte line (zero before the first call; left zero).
 struct IndexWsLayout {
-  size_t q_off, words_off, ticket_off, total;
+  size_t q_off, words_off, sync_off, total;
   int n_words;
 };
 
@@ -250,14 +551,14 @@ IndexWsLayout index_ws_layout(int B, int L, int max_cand) {
   IndexWsLayout s;
   s.n_words = (max_cand + 31) / 32;
   if (s.n_words < 1) s.n_words = 1;
-  // score CTAs write whole 256-row groups: round the word count up to 8-word groups
-  s.n_words = (s.n_words + 7) / 8 * 8;
   s.q_off = 0;
   s.words_off = align256(s.q_off + static_cast<size_t>(L) * B * lsa::idx::D_I * sizeof(float));
-  s.ticket_off = align256(s.words_off + static_cast<size_t>(B) * s.n_words * sizeof(uint32_t));
-  s.total = align256(s.ticket_off + static_cast<size_t>(B) * sizeof(int32_t));
+  s.sync_off = align256(s.words_off + static_cast<size_t>(B) * s.n_words * sizeof(uint32_t));
+  s.total = s.sync_off + 256;
   return s;
 }
+
+constexpr size_t kIndexSmem = sizeof(lsa::idx::Smem) + 128;   // + alignment slack
 }  // namespace
 
 extern "C" size_t lsa_index_workspace_size(int32_t B, int32_t L, int32_t d_i, int32_t max_cand) {
@@ -278,27 +579,34 @@ extern "C" lsa_status lsa_index(const uint16_t* h, const uint16_t* w_q, const fl
       D % 256 != 0 || max_cand < 0 || cap < 0)
     return LSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(h) | reinterpret_cast<uintptr_t>(w_q) |
-       reinterpret_cast<uintptr_t>(k_idx)) & 15u)
+       reinterpret_cast<uintptr_t>(k_idx) | reinterpret_cast<uintptr_t>(ws)) & 15u)
     return LSA_ERR_INVALID_ARG;
   const IndexWsLayout lay = index_ws_layout(B, L, max_cand);
   if (ws_bytes < lay.total) return LSA_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n_sm = lsa_host::sm_count();
+  if (n_sm <= 0) return LSA_ERR_CUDA;
+  const int G = n_sm < lsa::idx::MAX_GRID ? n_sm : lsa::idx::MAX_GRID;
+
+  static int configured_device = -1;   // the attribute is per device and function
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LSA_ERR_CUDA;
+  if (configured_device != dev) {
+    if (cudaFuncSetAttribute(lsa::idx::index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kIndexSmem)) != cudaSuccess)
+      return LSA_ERR_CUDA;
+    configured_device = dev;
+  }
   uint8_t* base = static_cast<uint8_t*>(ws);
-  float* q = reinterpret_cast<float*>(base + lay.q_off);
-
-  const int rows = L * lsa::idx::D_I;
-  lsa::idx::project_kernel<<<(rows + lsa::idx::PROJ_WARPS - 1) / lsa::idx::PROJ_WARPS,
-                             lsa::idx::PROJ_WARPS * 32, 0, s>>>(h, w_q, B, L, D, q);
-  if (cudaGetLastError() != cudaSuccess) return LSA_ERR_CUDA;
-
-  lsa::idx::ScoreArgs a;
+  lsa::idx::Args a;
+  a.h = h;
+  a.w_q = w_q;
+  a.bias = bias;
   a.k_idx = k_idx;
   a.kidx_off = kidx_off;
   a.n_cand = n_cand;
-  a.bias = bias;
-  a.q = q;
+  a.q = reinterpret_cast<float*>(base + lay.q_off);
   a.words = reinterpret_cast<uint32_t*>(base + lay.words_off);
-  a.ticket = reinterpret_cast<int32_t*>(base + lay.ticket_off);
+  a.sync = reinterpret_cast<unsigned int*>(base + lay.sync_off);
   a.sel_ids = sel_ids;
   a.sel_cnt = sel_cnt;
   a.logits = logits;
@@ -306,12 +614,28 @@ extern "C" lsa_status lsa_index(const uint16_t* h, const uint16_t* w_q, const fl
   a.err = err;
   a.B = B;
   a.L = L;
+  a.D = D;
   a.max_cand = max_cand;
   a.n_words = lay.n_words;
   a.mask_words = (max_cand + 31) / 32;
   a.cap = cap;
   a.inv_sqrt_di = 1.0f / sqrtf(static_cast<float>(d_i));
-  const int gx = max(1, (max_cand + lsa::idx::ROWS_PER_CTA - 1) / lsa::idx::ROWS_PER_CTA);
-  lsa::idx::score_kernel<<<dim3(gx, B), lsa::idx::SCORE_WARPS * 32, 0, s>>>(a);
-  return cudaGetLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+
+  // Cooperative launch: the G CTAs (one per SM) are resident together, which the two
+  // grid barriers rely on.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(lsa::idx::NTHREADS);
+  cfg.dynamicSmemBytes = kIndexSmem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, lsa::idx::index_kernel, a) != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
+  return LSA_OK;
 }

@@ -101,3 +101,43 @@ def test_all_and_none_kept(cuda_ok):
             assert ids[0, :int(cnt[0])].tolist() == list(range(n_cand[0]))
         else:
             assert int(cnt[0]) == 0
+
+
+def test_many_short_sequences(cuda_ok):
+    """Hundreds of sequences of 0..90 candidates: many sequences share a CTA's range of
+    keep words, some have none, word boundaries fall inside and between sequences."""
+    dev = torch.device("cuda")
+    g = torch.Generator().manual_seed(11)
+    B, L, D, d_i = 300, 3, 1024, 128
+    n_cand = torch.randint(0, 91, (B,), generator=g)
+    n_cand[::7] = 0
+    rows = int(n_cand.sum())
+    off = torch.zeros(B, dtype=torch.int64)
+    off[1:] = torch.cumsum(n_cand, 0)[:-1]
+    w_q = (torch.randn(L, d_i, D, generator=g) / D ** 0.5).to(torch.bfloat16)
+    h = torch.randn(L, B, D, generator=g).to(torch.bfloat16)
+    k_idx = torch.randn(max(1, rows), d_i, generator=g).to(torch.bfloat16)
+    bias = (torch.rand(B, generator=g) * 2.0 - 3.0).float()
+    max_cand = int(n_cand.max())
+    sel_ids = torch.full((B, max_cand), -1, dtype=torch.int32, device=dev)
+    sel_cnt = torch.full((B,), -1, dtype=torch.int32, device=dev)
+    logits = torch.full((L, B, max_cand), float("nan"), device=dev)
+    ws = torch.zeros(lsa.index_workspace_size(B, L, d_i, max_cand), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    wb, hb, kb = bits(w_q), bits(h), bits(k_idx)
+    for _ in range(2):      # the workspace is reusable as left
+        lsa.lsa_index(h.to(dev), w_q.to(dev), bias.to(dev), k_idx.to(dev), off.to(dev),
+                      n_cand.to(torch.int32).to(dev), max_cand, sel_ids, sel_cnt, ws, err,
+                      logits=logits)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        ids, cnt, z_gpu = sel_ids.cpu(), sel_cnt.cpu(), logits.cpu().numpy()
+        for b in range(B):
+            nc = int(n_cand[b])
+            ref_ids, z_ref = oracle.index_pass(wb, hb[:, b], kb[int(off[b]):int(off[b]) + nc],
+                                               float(bias[b]))
+            assert np.abs(z_gpu[:, b, :nc] - z_ref).max(initial=0.0) <= LOGIT_ABS
+            got = ids[b, :int(cnt[b])].tolist()
+            compare_selection(got, ref_ids, z_ref, "short b%d" % b)
+            assert got == np.flatnonzero((z_gpu[:, b, :nc] > 0).any(axis=0)).tolist()
+        assert not ws[-256:].any()      # barrier counters left at zero
