@@ -247,6 +247,27 @@ def attn_bytes_per_step(cfg, n_sel, s):
     return total
 
 
+def index_launch_ms(dec, inp, reps=20, rounds=5):
+    """Mean duration of one lsa_index launch: `reps` launches back to back in one CUDA
+    graph, replayed `rounds` times between two events (no event node between launches)."""
+    import torch
+    stream = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        for _ in range(reps):
+            dec.index(inp.h)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(rounds):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / (reps * rounds)
+
+
 def index_bytes(cfg, n_cand, n_sel):
     return (cfg.L * cfg.d_i * cfg.D * 2 + cfg.B * cfg.L * cfg.D * 2 + sum(n_cand) * cfg.d_i * 2
             + 4 * sum(n_sel))
@@ -528,7 +549,8 @@ def run_lsa(args, rank, world, local):
     achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
     traffic, traffic_src = profiled_traffic("attn_decode_step_1m_b20")
     ib = index_bytes(cfg, n_cand, n_sel)
-    idx_avg = statistics.mean(idx_ms)
+    idx_in_pass = statistics.mean(idx_ms)
+    idx_avg = index_launch_ms(dec, inp)
     gather_bytes = sum(n_sel) * 2 * 64 * cfg.d * 2
     gth_avg = statistics.mean(gth_ms)
     h2d_peak = pinned_h2d_gbs(dev)
@@ -552,7 +574,8 @@ def run_lsa(args, rank, world, local):
                      "traffic": traffic, "traffic_source": traffic_src,
                      "algorithmic_bytes_per_launch": attn_bytes,
                      "avg_launch_ms": attn_avg_ms},
-        "indexer": {"ms": idx_avg, "algorithmic_bytes": ib,
+        "indexer": {"ms": idx_avg, "timing": "20 launches back to back in one graph",
+                    "ms_in_pass": idx_in_pass, "algorithmic_bytes": ib,
                     "achieved_GBs": ib / (idx_avg * 1e-3) / 1e9,
                     "frac": ib / (idx_avg * 1e-3) / 1e9 / hbm, "kept_blocks": n_sel,
                     "candidates": n_cand},

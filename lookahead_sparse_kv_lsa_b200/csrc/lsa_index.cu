@@ -8,15 +8,16 @@
 //
 // One cooperative launch, one CTA per SM, three phases split by two grid barriers:
 //
-//  A. Each CTA starts 1-D bulk copies of its share of K_idx into shared memory (it does
-//     not depend on q), then computes its share of the W_q rows: q[l][b][j] = W_q[l][j] .
-//     h[l][b] in fp32, each dot cut into four fixed parts summed in a fixed order.
+//  A. Warp 0 starts 16-byte asynchronous copies of the CTA's share of K_idx into
+//     shared memory (it does not depend on q); warps 1.. compute the CTA's share of the
+//     W_q rows: q[l][b][j] = W_q[l][j] . h[l][b] in fp32, each dot cut into four fixed
+//     parts summed in a fixed order.
 //  B. Scoring. The candidate rows of every sequence are grouped in 32-row "words"; all
 //     words of the batch, in sequence order, are divided evenly over the CTAs. A warp
-//     scores one word from shared memory, 8 lanes per row (16 bytes of the row each, so
-//     the 4 rows a load instruction covers fall in disjoint banks):
-//     z_l = q_l . k / sqrt(d_i) + bias, keep bit z_l > 0 (equal to sigmoid(z_l) > 0.5),
-//     OR over the layers, collected into the word with warp ballots.
+//     scores one word from shared memory, one lane per row (rows padded by 16 bytes so
+//     the lanes' loads fall in different banks; the queries are broadcasts):
+//     z_l = q_l . k / sqrt(d_i) + bias, keep bit z_l > 0 (equal to sigmoid(z_l) > 0.5);
+//     one ballot per layer gives the word, OR-ed over the layers.
 //  C. Compaction. Each CTA ranks the kept bits of its words (popcounts of the earlier
 //     words of the same sequence, a block scan over its own) and writes the ascending id
 //     list; the CTA holding a sequence's last word writes its count.
@@ -34,8 +35,11 @@ constexpr int NTHREADS = 256;
 constexpr int NWARPS = NTHREADS / 32;
 constexpr int WORD_ROWS = 32;                       // candidate rows per keep word
 constexpr int ROW_BYTES = D_I * 2;                  // one K_idx row, bf16
-constexpr int WORD_BYTES = WORD_ROWS * ROW_BYTES;   // 8 KB
-constexpr int CHUNK_WORDS = 20;                     // K_idx words resident at once (160 KB)
+constexpr int ROW_STRIDE = ROW_BYTES + 16;          // padded row in shared memory: the
+                                                    // 16-byte pieces lanes read at once
+                                                    // fall in different banks
+constexpr int WORD_SMEM = WORD_ROWS * ROW_STRIDE;   // 8.5 KB
+constexpr int CHUNK_WORDS = 20;                     // K_idx words resident at once (170 KB)
 constexpr int NPART = 4;                            // projection: parts per dot product
 constexpr int RMAX = 4;                             // projection: W_q rows per round
 constexpr int BCH = 32;                             // projection: sequences per round
@@ -75,17 +79,17 @@ struct SeqTab {
 };
 
 struct Smem {
-  uint8_t kbuf[CHUNK_WORDS * WORD_BYTES];
-  uint64_t kbar;
+  uint8_t kbuf[CHUNK_WORDS * WORD_SMEM];
   int abort;
   int word_seq[CHUNK_WORDS];             // table entry of each word of the chunk
-  uint32_t wbits[MAX_L][CHUNK_WORDS];    // keep bits of the chunk's words, per layer
   alignas(16) float qs[CHUNK_WORDS][MAX_L][D_I];   // queries of the chunk's sequences
   int red[NWARPS];
   SeqTab tab;
   float part[RMAX][BCH][NPART];          // projection partial sums
   long long nw_total;
 };
+
+static_assert(sizeof(Smem) + 128 <= 227 * 1024, "shared memory per CTA");
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -199,38 +203,38 @@ __device__ __forceinline__ void grid_sync(const Args& a, Smem* s, unsigned int k
   __syncthreads();
 }
 
-// Warp 0: plan the chunk [cw0, cw1) of keep words and start the bulk copies of their
-// K_idx rows into s->kbuf (one copy per word; a sequence's last word may be partial).
+// Warp 0: plan the chunk [cw0, cw1) of keep words and start the 16-byte asynchronous
+// copies of their K_idx rows into s->kbuf (padded rows; a sequence's last word may be
+// partial). Completed by cp_async_wait_all in the same warp.
 __device__ __forceinline__ void issue_chunk(const Args& a, Smem* s, long long cw0, long long cw1,
                                             int lane) {
   plan_words(a, cw0, cw1, &s->tab, lane);
   __syncwarp();
   const int nwc = static_cast<int>(cw1 - cw0);
-  uint32_t bytes = 0;
-  const uint16_t* src = nullptr;
   if (lane < nwc) {
     const long long w = cw0 + lane;
     int i = 0;
     while (i + 1 < s->tab.n && s->tab.w0[i + 1] <= w) ++i;
-    const int wi = static_cast<int>(w - s->tab.w0[i]);
-    const int rows = min(WORD_ROWS, s->tab.nc[i] - WORD_ROWS * wi);
-    bytes = static_cast<uint32_t>(rows) * ROW_BYTES;
-    src = a.k_idx + (s->tab.row0[i] + static_cast<long long>(WORD_ROWS) * wi) * D_I;
     s->word_seq[lane] = i;
   }
-  uint32_t total = bytes;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
-  if (lane == 0) {
-    fence_proxy_async_smem();          // earlier generic reads of kbuf before the refill
-    mbar_arrive_expect_tx(&s->kbar, total);
-  }
   __syncwarp();
-  if (lane < nwc) bulk_load(s->kbuf + lane * WORD_BYTES, src, bytes, &s->kbar);
+  for (int k = 0; k < nwc; ++k) {
+    const int i = s->word_seq[k];
+    const int wi = static_cast<int>(cw0 + k - s->tab.w0[i]);
+    const int rows = min(WORD_ROWS, s->tab.nc[i] - WORD_ROWS * wi);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(
+        a.k_idx + (s->tab.row0[i] + static_cast<long long>(WORD_ROWS) * wi) * D_I);
+    const uint32_t dst = smem_u32(s->kbuf + k * WORD_SMEM);
+    for (int p = lane; p < rows * (ROW_BYTES / 16); p += 32) {
+      const int r = p >> 4, c = p & 15;
+      cp_async16(dst + r * ROW_STRIDE + c * 16, src + r * ROW_BYTES + c * 16);
+    }
+  }
+  cp_async_commit();
 }
 
-// All threads: stage the queries of the chunk's sequences in shared memory and clear
-// the chunk's keep bits (one round trip to L2 for the whole CTA).
+// All threads: stage the queries of the chunk's sequences in shared memory (one round
+// trip to L2 for the whole CTA).
 __device__ __forceinline__ void stage_queries(const Args& a, Smem* s) {
   const int per_seq = a.L * (D_I / 4);                  // float4s per sequence
   const int total = s->tab.n * per_seq;
@@ -241,82 +245,63 @@ __device__ __forceinline__ void stage_queries(const Args& a, Smem* s) {
                                 a.q + (static_cast<long long>(l) * a.B + s->tab.b[e]) * D_I) + c4);
     *reinterpret_cast<float4*>(&s->qs[e][l][4 * c4]) = v;
   }
-  for (int i = threadIdx.x; i < MAX_L * CHUNK_WORDS; i += NTHREADS) (&s->wbits[0][0])[i] = 0u;
 }
 
-// Warp: rows 4*st .. 4*st+3 of keep word k of the current chunk, 8 lanes per row (lane
-// sub reads 16-byte pieces sub and sub+8 of its row). The 4 keep bits of each layer go
-// into the word's bits in shared memory.
-__device__ __forceinline__ void score_rows(const Args& a, Smem* s, int k, int st, long long cw0,
-                                           int lane) {
+// Warp: keep word k of the current chunk, one lane per candidate row. The row's 16
+// pieces of 8 elements are read from its padded shared-memory row, the queries' pieces
+// are shared-memory broadcasts; each layer's dot product runs in two interleaved chains
+// joined in a fixed order. One ballot per layer gives the word's keep bits.
+__device__ __forceinline__ void score_word(const Args& a, Smem* s, int k, long long cw0, int lane) {
   const int i = s->word_seq[k];
   const int wi = static_cast<int>(cw0 + k - s->tab.w0[i]);
-  const int n = s->tab.nc[i];
+  const int c = WORD_ROWS * wi + lane;
+  const bool valid = c < s->tab.nc[i];
   const float bias = s->tab.bias[i];
-  const int sub = lane & 7;
-  const int rl = 4 * st + (lane >> 3);
-  const int c = WORD_ROWS * wi + rl;
-  const bool valid = c < n;
-  const uint8_t* rp = s->kbuf + k * WORD_BYTES + rl * ROW_BYTES + 16 * sub;
-  float k0[8], k1[8];
-  unpack8(*reinterpret_cast<const uint4*>(rp), k0);
-  unpack8(*reinterpret_cast<const uint4*>(rp + 128), k1);
-  float z[MAX_L];
-#pragma unroll
-  for (int l = 0; l < MAX_L; ++l) {
-    if (l < a.L) {
-      const float4* q0 = reinterpret_cast<const float4*>(&s->qs[i][l][8 * sub]);
-      const float4* q1 = reinterpret_cast<const float4*>(&s->qs[i][l][64 + 8 * sub]);
-      const float4 qa = q0[0], qb = q0[1], qc = q1[0], qd = q1[1];
-      // two independent chains, joined in a fixed order
-      float u = qa.x * k0[0], v = qc.x * k1[0];
-      u = fmaf(qa.y, k0[1], u); v = fmaf(qc.y, k1[1], v);
-      u = fmaf(qa.z, k0[2], u); v = fmaf(qc.z, k1[2], v);
-      u = fmaf(qa.w, k0[3], u); v = fmaf(qc.w, k1[3], v);
-      u = fmaf(qb.x, k0[4], u); v = fmaf(qd.x, k1[4], v);
-      u = fmaf(qb.y, k0[5], u); v = fmaf(qd.y, k1[5], v);
-      u = fmaf(qb.z, k0[6], u); v = fmaf(qd.z, k1[6], v);
-      u = fmaf(qb.w, k0[7], u); v = fmaf(qd.w, k1[7], v);
-      z[l] = u + v;
-    }
-  }
-#pragma unroll
-  for (int o = 4; o >= 1; o >>= 1) {
-#pragma unroll
-    for (int l = 0; l < MAX_L; ++l)
-      if (l < a.L) z[l] += __shfl_xor_sync(0xffffffffu, z[l], o);
-  }
   const int b = s->tab.b[i];
+  const uint8_t* rp = s->kbuf + k * WORD_SMEM + lane * ROW_STRIDE;
+  float acc[MAX_L][2];
 #pragma unroll
-  for (int l = 0; l < MAX_L; ++l) {
-    if (l < a.L) {
-      const float zz = fmaf(z[l], a.inv_sqrt_di, bias);
-      const bool keep = valid && zz > 0.f;
-      if (a.logits != nullptr && sub == 0 && valid)
-        a.logits[(static_cast<long long>(l) * a.B + b) * a.max_cand + c] = zz;
-      const uint32_t bal = __ballot_sync(0xffffffffu, keep && sub == 0);
-      const uint32_t nib = (bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u);
-      if (lane == 0 && nib != 0u) atomicOr(&s->wbits[l][k], nib << (4 * st));
+  for (int l = 0; l < MAX_L; ++l) acc[l][0] = acc[l][1] = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < D_I / 8; ++j) {
+    float kf[8];
+    unpack8(*reinterpret_cast<const uint4*>(rp + 16 * j), kf);
+#pragma unroll
+    for (int l = 0; l < MAX_L; ++l) {
+      if (l < a.L) {
+        const float4 qa = *reinterpret_cast<const float4*>(&s->qs[i][l][8 * j]);
+        const float4 qb = *reinterpret_cast<const float4*>(&s->qs[i][l][8 * j + 4]);
+        float& u = acc[l][j & 1];
+        u = fmaf(qa.x, kf[0], u);
+        u = fmaf(qa.y, kf[1], u);
+        u = fmaf(qa.z, kf[2], u);
+        u = fmaf(qa.w, kf[3], u);
+        u = fmaf(qb.x, kf[4], u);
+        u = fmaf(qb.y, kf[5], u);
+        u = fmaf(qb.z, kf[6], u);
+        u = fmaf(qb.w, kf[7], u);
+      }
     }
   }
-}
-
-// Threads: write the chunk's keep words (OR over the layers, and the per-layer masks).
-__device__ __forceinline__ void store_words(const Args& a, Smem* s, int nwc, long long cw0) {
-  for (int k = threadIdx.x; k < nwc; k += NTHREADS) {
-    const int i = s->word_seq[k];
-    const int b = s->tab.b[i];
-    const int wi = static_cast<int>(cw0 + k - s->tab.w0[i]);
-    uint32_t wor = 0;
+  uint32_t wor = 0;
+  uint32_t wl[MAX_L];
 #pragma unroll
-    for (int l = 0; l < MAX_L; ++l)
-      if (l < a.L) wor |= s->wbits[l][k];
+  for (int l = 0; l < MAX_L; ++l) {
+    wl[l] = 0u;
+    if (l < a.L) {
+      const float z = fmaf(acc[l][0] + acc[l][1], a.inv_sqrt_di, bias);
+      if (a.logits != nullptr && valid)
+        a.logits[(static_cast<long long>(l) * a.B + b) * a.max_cand + c] = z;
+      wl[l] = __ballot_sync(0xffffffffu, valid && z > 0.f);
+      wor |= wl[l];
+    }
+  }
+  if (lane == 0) {
     a.words[static_cast<long long>(b) * a.n_words + wi] = wor;
     if (a.layer_mask != nullptr) {
 #pragma unroll
       for (int l = 0; l < MAX_L; ++l)
-        if (l < a.L)
-          a.layer_mask[(static_cast<long long>(l) * a.B + b) * a.mask_words + wi] = s->wbits[l][k];
+        if (l < a.L) a.layer_mask[(static_cast<long long>(l) * a.B + b) * a.mask_words + wi] = wl[l];
       a.layer_mask[(static_cast<long long>(a.L) * a.B + b) * a.mask_words + wi] = wor;
     }
   }
@@ -432,11 +417,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
   const int cta = blockIdx.x;
 
   if (tid == 0) {
-    mbar_init(&s->kbar, 1);
     s->abort = 0;
     s->tab.resume_b = 0;
     s->tab.resume_base = 0;
-    fence_barrier_init();
   }
   __syncthreads();
   // ---- phase A. Warp 0: this CTA's keep words [W0, W1), whose first chunk of K_idx
@@ -454,31 +437,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
   const long long NW = s->nw_total;
   const long long W0 = (cta * NW) / G, W1 = ((cta + 1) * NW) / G;
 
-  // ---- phase B: keep words
-  uint32_t parity = 0;
+  // ---- phase B: keep words, one warp per word
   for (long long cw0 = W0; cw0 < W1; cw0 += CHUNK_WORDS) {
     const long long cw1 = W1 < cw0 + CHUNK_WORDS ? W1 : cw0 + CHUNK_WORDS;
     if (cw0 != W0) {
       __syncthreads();                          // every warp is done with kbuf
       if (warp == 0) issue_chunk(a, s, cw0, cw1, lane);
-      __syncthreads();
+      __syncthreads();                          // the chunk's plan is visible
     }
-    // always wait for the copies in flight, even after an abort (bounded)
-    const bool landed = mbar_wait(&s->kbar, parity, nullptr);
-    parity ^= 1u;
-    if (!landed && tid == 0) {
-      set_err(a.err, LSA_DEVERR_TIMEOUT);
-      s->abort = 1;
-    }
+    if (warp == 0) cp_async_wait_all();         // the chunk's rows (issued by warp 0)
     if (!s->abort) stage_queries(a, s);
     __syncthreads();
     if (s->abort) break;
-    // tasks (word, 4-row step) round-robin over the warps: a warp's tasks are independent
     const int nwc = static_cast<int>(cw1 - cw0);
-    for (int t = warp; t < nwc * (WORD_ROWS / 4); t += NWARPS)
-      score_rows(a, s, t >> 3, t & 7, cw0, lane);
-    __syncthreads();
-    store_words(a, s, nwc, cw0);
+    for (int k = warp; k < nwc; k += NWARPS) score_word(a, s, k, cw0, lane);
   }
   grid_sync(a, s, 2);
 
