@@ -75,7 +75,7 @@ struct Args {
   const int32_t* block_table;
   const int32_t* n_entries;
   const int32_t* tail_len;
-  float* part_o;          // [slots][H][d] fp32
+  float* part_o;          // [slots][d/128][H][128] fp32: each 128-dim block contiguous
   float* part_ml;         // [slots][H][2] fp32 (running max in log2 units, denominator)
   unsigned int* sync;     // [2] grid-barrier arrive / depart counters (left at zero)
   uint16_t* out;          // [B][H][d] bf16
@@ -462,7 +462,8 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
         if (r0 < rows_per_pass) {
           const long long b = m->run_b[q], h = m->run_h[q];
           const uint32_t dst0 = smem_u32(buf + m->run_off[q]) + c * 16;
-          const float* src0 = a.part_o + (h * a.d + m->run_d0[q] + 4 * c);
+          const int x = m->run_d0[q] + 4 * c;       // head dimension of this column
+          const float* src0 = a.part_o + ((x >> 7) * a.H + h) * 128 + (x & 127);
           for (int k = r0; k < n; k += rows_per_pass) {
             const long long slot = m->run_clo[q] + k + b;
             cp_async16(dst0 + static_cast<uint32_t>(k) * (w4 * 16),
@@ -991,12 +992,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
-            if (t128 < a.H) {
-              const uint8_t* src = smem + db * blk_bytes + t128 * 128 * esz;
-              if (whole)
+            if (whole) {
+              if (t128 < a.H) {
+                const uint8_t* src = smem + db * blk_bytes + t128 * 256;
                 bulk_store(fo + static_cast<long long>(t128) * a.d + db * 128, src, 256u);
-              else
-                bulk_store(po + static_cast<long long>(t128) * a.d + db * 128, src, 512u);
+                issued = true;
+              }
+            } else if (t128 == 0) {
+              // the partial's block db is [H][128] in both places: one copy
+              bulk_store(po + static_cast<long long>(db) * a.H * 128, smem + db * blk_bytes, blk_bytes);
               issued = true;
             }
           } else if (whole) {
@@ -1007,9 +1011,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 fo[static_cast<long long>(h) * a.d + col] = *reinterpret_cast<const uint16_t*>(&v);
               }
           } else {
+            float* pb = po + static_cast<long long>(db) * a.H * 128 + row;
 #pragma unroll
             for (int h = 0; h < HP; ++h)
-              if (h < a.H) po[static_cast<long long>(h) * a.d + col] = ob[h];
+              if (h < a.H) pb[h * 128] = ob[h];
           }
         }
         if (issued) {
@@ -1068,7 +1073,7 @@ namespace {
 using lsa::attn::Args;
 
 // Workspace: the two grid-barrier counters on their own 256-byte line, then fp32
-// partial O [G+B][H][d] and partial (m, l) [G+B][H][2].
+// partial O [G+B][d/128][H][128] and partial (m, l) [G+B][H][2].
 size_t attn_ws_bytes(int B, int H, int d, int n_sm) {
   const size_t slots = static_cast<size_t>(n_sm) + static_cast<size_t>(B);
   const size_t body = slots * static_cast<size_t>(H) * (static_cast<size_t>(d) + 2) * sizeof(float);
