@@ -42,7 +42,7 @@ DEFAULT_WORKLOAD = "1m_b20"
 FALLBACK_HBM_GBS = 6650.0
 LAUNCHES_PER_DECODE_STEP = 1      # one fused kernel: append + split-K attention + merge
 LAUNCHES_PER_PASS_HEAD = 4        # pass set-up, projection, scoring, gather
-SEL_PAGES = 4096                  # HBM pages for kept blocks (1,079 used at bias -2; 512 MB)
+SEL_PAGES_CAP = 65536             # HBM pages for kept blocks at most (8 GB at d = 512)
 
 
 def parse_args():
@@ -75,11 +75,17 @@ def peaks():
 
 
 def workload_desc(cfg):
-    return ("%s: B=%d, context %d tokens (%d blocks of 64), window %d, %d heads x d %d MQA, "
-            "3 indexer layers D=%d, bias %s" % (cfg.name, cfg.B, cfg.ctx_tokens[0] if cfg.ctx_tokens
-                                                else -1, (cfg.ctx_tokens[0] // 64) if cfg.ctx_tokens
-                                                else -1, cfg.W, cfg.H, cfg.d, cfg.D,
-                                                cfg.bias[0] if cfg.bias else "ragged"))
+    if cfg.ctx_tokens:
+        ctx = "context %d tokens (%d blocks of 64)" % (cfg.ctx_tokens[0], cfg.ctx_tokens[0] // 64)
+    else:
+        lo, hi = cfg.ctx_uniform_blocks
+        ctx = "context U{%d..%d} blocks of 64 per sequence" % (lo, hi)
+    if cfg.bias:
+        bias = "bias %s" % cfg.bias[0]
+    else:
+        bias = "bias U(%g, %g) per sequence" % cfg.bias_uniform
+    return ("%s: B=%d, %s, window %d, %d heads x d %d MQA, 3 indexer layers D=%d, %s"
+            % (cfg.name, cfg.B, ctx, cfg.W, cfg.H, cfg.d, cfg.D, bias))
 
 
 # ----------------------------------------------------------------------- clocks
@@ -189,7 +195,7 @@ def make_decoder(wl, dev):
     dec = lsa.LsaDecoder(wl.w_q.to(dev), wl.k_idx.to(dev), wl.blk_off[:c.B],
                          torch.from_numpy(wl.bias).to(dev), wl.host_pool, wl.blk_off, wl.nb0,
                          W=c.W, H=c.H, cap=max_cand, max_cand=max_cand, scale=c.scale,
-                         sel_pages=min(c.B * max_cand, SEL_PAGES))
+                         sel_pages=min(c.B * max_cand, SEL_PAGES_CAP))
     dec.load_window(0)
     return dec, n_cand
 
@@ -236,13 +242,12 @@ def event_breakdown(evs, tau):
     return idx, gth, step
 
 
-def attn_bytes_per_step(cfg, n_sel, s):
+def attn_bytes_per_step(cfg, ctx, n_sel, s):
     """Algorithmic bytes of one decode-attention launch: K and V of the attended tokens,
-    q in and out (bf16)."""
+    q in and out (bf16). ctx: tokens of each sequence when the pass starts."""
     total = 0
     for b in range(cfg.B):
-        T = n_sel[b] * cfg.block + min(cfg.W, int(cfg.ctx_tokens[b]) if cfg.ctx_tokens else
-                                        cfg.W) + s + 1
+        T = n_sel[b] * cfg.block + min(cfg.W, int(ctx[b])) + s + 1
         total += 2 * cfg.d * 2 * T + 2 * cfg.H * cfg.d * 2
     return total
 
@@ -335,9 +340,17 @@ def oracle_threads():
         return 1
 
 
+def sample_sequences(B, k=4):
+    """At most k sequences spread over the batch (the oracle is timed on these)."""
+    if B <= k:
+        return list(range(B))
+    return sorted({(i * (B - 1)) // (k - 1) for i in range(k)})
+
+
 def oracle_pass_seconds(wl, steps):
-    """Time the CPU oracle on one indexer pass and on the given decode steps of pass 0;
-    returns (seconds for the whole 64-step pass, extrapolated, seconds actually spent)."""
+    """Time the CPU oracle on one indexer pass and on the given decode steps of pass 0 for
+    a sample of the batch's sequences; returns (seconds for the whole batch's 64-step
+    pass, extrapolated over steps and sequences, seconds actually spent)."""
     import oracle
     from lsa_inputs import bf16_bits
     c = wl.cfg
@@ -345,7 +358,8 @@ def oracle_pass_seconds(wl, steps):
     t_idx, t_steps = 0.0, []
     hb = bf16_bits(wl.h(0))
     wq = bf16_bits(wl.w_q)
-    for b in range(c.B):
+    seqs = sample_sequences(c.B)
+    for b in seqs:
         n_ctx = int(wl.ctx_at(0)[b])
         nc = oracle.n_candidates(n_ctx, c.W)
         t0 = time.perf_counter()
@@ -358,8 +372,9 @@ def oracle_pass_seconds(wl, steps):
             t0 = time.perf_counter()
             oracle.step_output(qb, Kb, Vb, ids, n_ctx, c.W, s, c.scale)
             t_steps.append(time.perf_counter() - t0)
-    per_step = sum(t_steps) / max(1, len(steps))      # summed over the batch
-    return t_idx + c.tau * per_step, time.perf_counter() - t_start
+    per_step = sum(t_steps) / max(1, len(steps))      # summed over the sampled sequences
+    scale = c.B / len(seqs)
+    return scale * (t_idx + c.tau * per_step), time.perf_counter() - t_start
 
 
 def cpu_baseline(wl, steps=tuple(range(64))):
@@ -367,9 +382,9 @@ def cpu_baseline(wl, steps=tuple(range(64))):
     t_pass, spent = oracle_pass_seconds(wl, steps)
     return {"value": c.B * c.tau / t_pass, "unit": UNIT, "cores": oracle_threads(),
             "kind": "oracle",
-            "sample": "float64 numpy oracle: one indexer pass + decode steps %s of pass 0 of %s, "
-                      "extrapolated to the 64-step pass (%.1f s of CPU work)"
-                      % (list(steps), c.name, spent)}
+            "sample": "float64 numpy oracle: one indexer pass + decode steps %s of pass 0 of %s "
+                      "for sequences %s, extrapolated to the batch's 64-step pass (%.1f s of "
+                      "CPU work)" % (list(steps), c.name, sample_sequences(c.B), spent)}
 
 
 def run_reference(args, rank, world):
@@ -497,8 +512,6 @@ def run_lsa(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     cfg = LI.by_name(args.workload)
-    if cfg.ctx_tokens is None:
-        raise SystemExit("bench workloads have a fixed context length")
     wl = LI.Workload(cfg, pin=True)
     dec, n_cand = make_decoder(wl, dev)
     inp = Inputs(wl, dev)
@@ -544,7 +557,8 @@ def run_lsa(args, rank, world, local):
         a, g, at = event_breakdown(events[i], cfg.tau)
         idx_ms.append(a); gth_ms.append(g); attn_ms.append(at)
     hbm, peak_src = peaks()
-    attn_bytes = sum(attn_bytes_per_step(cfg, n_sel, s) for s in range(cfg.tau)) / cfg.tau
+    attn_bytes = sum(attn_bytes_per_step(cfg, wl.ctx_at(0), n_sel, s)
+                     for s in range(cfg.tau)) / cfg.tau
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
     traffic, traffic_src = profiled_traffic("attn_decode_step_1m_b20")
@@ -599,7 +613,9 @@ def run_lsa(args, rank, world, local):
     if not args.no_e2e:
         line["e2e"] = e2e_measure(dec, wl, dev, args.steps, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl)
+        # the default workload samples all 64 steps; the others four of them
+        steps = tuple(range(cfg.tau)) if cfg.name == DEFAULT_WORKLOAD else (0, 21, 42, 63)
+        line["cpu_baseline"] = cpu_baseline(wl, steps)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
