@@ -889,8 +889,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float al = m->alpha[h];
             rescale |= al < 1.f;
             const float p = (valid && h < a.H) ? exp2f(fmaf(s[h], a.scale_log2, -mu)) : 0.f;
-            lp[h] = lp[h] * al + p;
-            s[h] = p;
+            // the denominator sums the same bf16-rounded weights that multiply V, so the
+            // output stays a normalised average of V rows (exact for a one-hot softmax)
+            const float pr = __bfloat162float(__float2bfloat16_rn(p));
+            lp[h] = lp[h] * al + pr;
+            s[h] = pr;
           }
           // the previous tile's P . V must be done before P is overwritten or O rescaled
           if (gtile_o >= 1)
