@@ -81,10 +81,15 @@ def block_logits(q: np.ndarray, k_idx: np.ndarray, bias: float) -> np.ndarray:
     """z_l[c] = q_l . K_idx[c] / sqrt(d_i) + bias, for every layer l and block c.
 
     q: [L][d_i]; k_idx: [n][d_i] (one frozen compressed key per candidate block,
-    shared by the layers). returns z: [L][n]. Scoring of step 3 of section 2.
+    shared by the layers) or [L][n][d_i] (each indexer layer with its own keys: the
+    "three small projection matrices" of section 3 paired with per-layer key tables).
+    returns z: [L][n]. Scoring of step 3 of section 2.
     """
-    d_i = k_idx.shape[1]
+    d_i = k_idx.shape[-1]
     assert q.shape[1] == d_i
+    if k_idx.ndim == 3:
+        assert k_idx.shape[0] == q.shape[0]
+        return np.stack([k_idx[l] @ q[l] for l in range(q.shape[0])]) / math.sqrt(d_i) + bias
     return (q @ k_idx.T) / math.sqrt(d_i) + bias
 
 
@@ -102,8 +107,9 @@ def kept_blocks(z: np.ndarray) -> np.ndarray:
 def index_pass(w_q_bits, h_bits, k_idx_bits, bias: float):
     """One indexer pass for one sequence.
 
-    w_q_bits [L][d_i][D], h_bits [L][D], k_idx_bits [n_cand][d_i] (bf16 bit patterns
-    of the candidate blocks only). Returns (ids, z) with z float64 [L][n_cand].
+    w_q_bits [L][d_i][D], h_bits [L][D], k_idx_bits [n_cand][d_i] or, with per-layer
+    keys, [L][n_cand][d_i] (bf16 bit patterns of the candidate blocks only). Returns
+    (ids, z) with z float64 [L][n_cand].
     """
     q = query_projection(bf16_to_f64(w_q_bits), bf16_to_f64(h_bits))
     z = block_logits(q, bf16_to_f64(k_idx_bits), float(bias))

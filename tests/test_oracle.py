@@ -238,8 +238,29 @@ def check_special_cases_reduce_to_dense(O=O):
     assert np.max(np.abs(got - win)) < 1e-12
 
 
+def check_per_layer_keys(O=O):
+    """Per-layer key tables: layer l scores against its own table (closed form), and
+    identical tables reduce to the shared-key case."""
+    d_i, n = 64, 7                     # sqrt(d_i) = 8 exactly
+    q = np.zeros((3, d_i))
+    q[:, 0] = [2.0, -1.0, 0.5]
+    k = np.zeros((3, n, d_i))
+    for l in range(3):
+        k[l, :, 0] = (np.arange(n) - 3.0) * (l + 1)      # table l = (l + 1) x base
+    bias = -0.125
+    z = O.block_logits(q, k, bias)
+    for l in range(3):
+        for c in range(n):
+            assert z[l, c] == q[l, 0] * (c - 3.0) * (l + 1) / 8.0 + bias
+    rng = np.random.default_rng(5)
+    qr = rng.standard_normal((3, 128))
+    kr = rng.standard_normal((11, 128))
+    same = O.block_logits(qr, np.stack([kr, kr, kr]), -2.0)
+    assert np.allclose(same, O.block_logits(qr, kr, -2.0), rtol=1e-13, atol=1e-13)
+
+
 PINS = [check_bf16_decode, check_projection_unit_rows, check_projection_bruteforce,
-        check_logits_closed_form, check_threshold_strict, check_union_bruteforce,
+        check_logits_closed_form, check_per_layer_keys, check_threshold_strict, check_union_bruteforce,
         check_selection_rate, check_single_token, check_two_token_closed_form,
         check_matches_sdpa, check_uniform_when_q_zero, check_attended_set,
         check_special_cases_reduce_to_dense]
@@ -313,6 +334,10 @@ MUTANTS = {
     "logit_no_bias": dict(block_logits=lambda q, k, b: (q @ k.T) / math.sqrt(k.shape[1])),
     "logit_no_scale": dict(block_logits=lambda q, k, b: (q @ k.T) + b),
     "logit_sqrt_of_wrong_dim": dict(block_logits=lambda q, k, b: (q @ k.T) / math.sqrt(q.shape[0]) + b),
+    "per_layer_keys_shifted": dict(block_logits=lambda q, k, b: O.block_logits(
+        q, k if k.ndim == 2 else np.roll(k, 1, axis=0), b)),
+    "per_layer_keys_first_table_only": dict(block_logits=lambda q, k, b: O.block_logits(
+        q, k if k.ndim == 2 else k[0], b)),
     "threshold_ge": dict(kept_blocks=lambda z: np.flatnonzero((z >= 0).any(axis=0))),
     "and_instead_of_or": dict(kept_blocks=lambda z: np.flatnonzero((z > 0).all(axis=0))),
     "only_first_layer": dict(kept_blocks=lambda z: np.flatnonzero(z[0] > 0)),
