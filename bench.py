@@ -274,8 +274,9 @@ def index_launch_ms(dec, inp, reps=20, rounds=5):
 
 
 def index_bytes(cfg, n_cand, n_sel):
-    return (cfg.L * cfg.d_i * cfg.D * 2 + cfg.B * cfg.L * cfg.D * 2 + sum(n_cand) * cfg.d_i * 2
-            + 4 * sum(n_sel))
+    tables = cfg.L if cfg.kidx_per_layer else 1     # compressed key tables read per block
+    return (cfg.L * cfg.d_i * cfg.D * 2 + cfg.B * cfg.L * cfg.D * 2
+            + tables * sum(n_cand) * cfg.d_i * 2 + 4 * sum(n_sel))
 
 
 def pinned_h2d_gbs(dev, nbytes=1 << 30):
@@ -363,7 +364,9 @@ def oracle_pass_seconds(wl, steps):
         n_ctx = int(wl.ctx_at(0)[b])
         nc = oracle.n_candidates(n_ctx, c.W)
         t0 = time.perf_counter()
-        ids, _ = oracle.index_pass(wq, hb[:, b], bf16_bits(wl.seq_k_idx(b)[:nc]), float(wl.bias[b]))
+        kb = wl.seq_k_idx(b)
+        kb = kb[:, :nc] if kb.dim() == 3 else kb[:nc]
+        ids, _ = oracle.index_pass(wq, hb[:, b], bf16_bits(kb), float(wl.bias[b]))
         t_idx += time.perf_counter() - t0
         K, V = wl.seq_kv(b)
         Kb, Vb = bf16_bits(K), bf16_bits(V)

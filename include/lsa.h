@@ -98,6 +98,27 @@ lsa_status lsa_index(const uint16_t* h, const uint16_t* w_q, const float* bias,
                      void* ws, size_t ws_bytes, int32_t* err, void* stream);
 size_t lsa_index_workspace_size(int32_t B, int32_t L, int32_t d_i, int32_t max_cand);
 
+/* lsa_index_ex -- lsa_index where each indexer layer may score against its own frozen
+ * compressed key table (section 3 of "FlashMemory-DeepSeek-V4 Explained": one small query
+ * encoder per indexer layer against precomputed block keys; per-layer tables are the
+ * reading where every indexer layer has its own keys):
+ *
+ *   z_l[b][c] = q_l . K_idx[l * kidx_layer_stride + kidx_off[b] + c] / sqrt(d_i) + bias[b]
+ *
+ *   kidx_layer_stride  rows between consecutive layers' tables in k_idx (each table laid
+ *                      out like the shared one, sequence b's blocks from kidx_off[b]);
+ *                      0 = one table shared by all layers (exactly lsa_index).
+ * Every other argument, the workspace and the errors are as for lsa_index. Per-layer
+ * tables read L x 256 bytes per candidate block instead of 256.
+ */
+lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const float* bias,
+                        const uint16_t* k_idx, int64_t kidx_layer_stride,
+                        const int64_t* kidx_off, const int32_t* n_cand,
+                        int32_t B, int32_t L, int32_t D, int32_t d_i, int32_t max_cand,
+                        int32_t* sel_ids, int32_t* sel_cnt, int32_t cap,
+                        float* logits, uint32_t* layer_mask,
+                        void* ws, size_t ws_bytes, int32_t* err, void* stream);
+
 /* ---------------------------------------------------------------------------------
  * lsa_gather -- move the kept blocks from the host cold pool into the HBM pool
  * (section 2 step 3) and build each sequence's block table.
@@ -248,6 +269,8 @@ typedef struct lsa_state {
   void* index_ws; size_t index_ws_bytes;   /* lsa_index_workspace_size(B, L, d_i, max_cand) */
   void* attn_ws;  size_t attn_ws_bytes;    /* lsa_decode_attn_workspace_size(B, H, d, n_sm) */
   int32_t* err;                        /* device i32 error word */
+  int64_t kidx_layer_stride;           /* 0: K_idx shared by the layers; > 0: rows from
+                                          layer l's key table to layer l+1's (lsa_index_ex) */
 } lsa_state;
 
 /* Host-side validation of a state (no device work). */

@@ -60,13 +60,21 @@ def decode_attn_workspace_size(B: int, H: int, d: int, n_sm: Optional[int] = Non
 
 def lsa_index(h, w_q, bias, k_idx, kidx_off, n_cand, max_cand: int, sel_ids, sel_cnt, ws, err,
               logits=None, layer_mask=None, stream=None) -> None:
-    """One indexer pass; see lsa_index in include/lsa.h. h [L][B][D], w_q [L][d_i][D]."""
+    """One indexer pass; see lsa_index / lsa_index_ex in include/lsa.h. h [L][B][D],
+    w_q [L][d_i][D]; k_idx [rows][d_i] (shared by the layers) or [L][rows][d_i] (one
+    table per layer)."""
     L, B, D = h.shape
     d_i = w_q.shape[1]
     cap = sel_ids.shape[1] if sel_ids.dim() == 2 else 0
-    st = _lib.lib().lsa_index(
+    if k_idx.dim() == 3:
+        if k_idx.shape[0] != L:
+            raise ValueError("per-layer k_idx must have L = %d tables" % L)
+        layer_stride = k_idx.shape[1]
+    else:
+        layer_stride = 0
+    st = _lib.lib().lsa_index_ex(
         _dev(h, torch.bfloat16, "h"), _dev(w_q, torch.bfloat16, "w_q", L * d_i * D),
-        _dev(bias, torch.float32, "bias", B), _dev(k_idx, torch.bfloat16, "k_idx"),
+        _dev(bias, torch.float32, "bias", B), _dev(k_idx, torch.bfloat16, "k_idx"), layer_stride,
         _dev(kidx_off, torch.int64, "kidx_off", B), _dev(n_cand, torch.int32, "n_cand", B),
         B, L, D, d_i, max_cand,
         _dev(sel_ids, torch.int32, "sel_ids"), _dev(sel_cnt, torch.int32, "sel_cnt", B), cap,

@@ -43,6 +43,7 @@ class LsaState(C.Structure):
         ("index_ws", _p), ("index_ws_bytes", _sz),
         ("attn_ws", _p), ("attn_ws_bytes", _sz),
         ("err", _p),
+        ("kidx_layer_stride", _i64),
     ]
 
 
@@ -52,6 +53,8 @@ SIGNATURES = {
     "lsa_version": (_i32, []),
     "lsa_index": (_i32, [_p, _p, _p, _p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _i32,
                          _p, _p, _p, _sz, _p, _p]),
+    "lsa_index_ex": (_i32, [_p, _p, _p, _p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p,
+                            _i32, _p, _p, _p, _sz, _p, _p]),
     "lsa_index_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
     "lsa_gather": (_i32, [_p, _i64, _p, _p, _p, _i32, _p, _p, _i32, _i32, _i32, _p, _i64, _i32,
                           _i32, _p, _i32, _p, _p, _p]),

@@ -370,9 +370,10 @@ extern "C" lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t
     if (!h) return LSA_ERR_INVALID_ARG;
     v = lsa_pass_setup(st, p, stream);
     if (v != LSA_OK) return v;
-    v = lsa_index(h, st->w_q, st->bias, st->k_idx, st->kidx_off, st->n_cand, st->B, st->L, st->D,
-                  st->d_i, st->max_cand, st->sel_ids, st->sel_cnt, st->cap, nullptr, nullptr,
-                  st->index_ws, st->index_ws_bytes, st->err, stream);
+    v = lsa_index_ex(h, st->w_q, st->bias, st->k_idx, st->kidx_layer_stride, st->kidx_off,
+                     st->n_cand, st->B, st->L, st->D, st->d_i, st->max_cand, st->sel_ids,
+                     st->sel_cnt, st->cap, nullptr, nullptr, st->index_ws, st->index_ws_bytes,
+                     st->err, stream);
     if (v != LSA_OK) return v;
     const int wb1 = st->W / LSA_BLOCK + 1;
     const int64_t base = static_cast<int64_t>(st->B) * wb1;

@@ -49,7 +49,9 @@ struct Args {
   const uint16_t* h;         // [L][B][D]
   const uint16_t* w_q;       // [L][D_I][D]
   const float* bias;         // [B]
-  const uint16_t* k_idx;     // [rows][D_I]
+  const uint16_t* k_idx;     // [rows][D_I]; table t of per-layer keys at row t * kls
+  long long kls;             // rows between the per-layer key tables (0: one shared table)
+  int lk;                    // key tables read per candidate: 1 (shared) or L
   const int64_t* kidx_off;   // [B]
   const int32_t* n_cand;     // [B]
   float* q;                  // workspace [L][B][D_I]
@@ -222,12 +224,14 @@ __device__ __forceinline__ void issue_chunk(const Args& a, Smem* s, long long cw
     const int i = s->word_seq[k];
     const int wi = static_cast<int>(cw0 + k - s->tab.w0[i]);
     const int rows = min(WORD_ROWS, s->tab.nc[i] - WORD_ROWS * wi);
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(
-        a.k_idx + (s->tab.row0[i] + static_cast<long long>(WORD_ROWS) * wi) * D_I);
-    const uint32_t dst = smem_u32(s->kbuf + k * WORD_SMEM);
-    for (int p = lane; p < rows * (ROW_BYTES / 16); p += 32) {
-      const int r = p >> 4, c = p & 15;
-      cp_async16(dst + r * ROW_STRIDE + c * 16, src + r * ROW_BYTES + c * 16);
+    for (int t = 0; t < a.lk; ++t) {       // the word's rows of each key table
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(
+          a.k_idx + (t * a.kls + s->tab.row0[i] + static_cast<long long>(WORD_ROWS) * wi) * D_I);
+      const uint32_t dst = smem_u32(s->kbuf + (k * a.lk + t) * WORD_SMEM);
+      for (int p = lane; p < rows * (ROW_BYTES / 16); p += 32) {
+        const int r = p >> 4, c = p & 15;
+        cp_async16(dst + r * ROW_STRIDE + c * 16, src + r * ROW_BYTES + c * 16);
+      }
     }
   }
   cp_async_commit();
@@ -251,6 +255,7 @@ __device__ __forceinline__ void stage_queries(const Args& a, Smem* s) {
 // pieces of 8 elements are read from its padded shared-memory row, the queries' pieces
 // are shared-memory broadcasts; each layer's dot product runs in two interleaved chains
 // joined in a fixed order. One ballot per layer gives the word's keep bits.
+template <bool PER_LAYER>
 __device__ __forceinline__ void score_word(const Args& a, Smem* s, int k, long long cw0, int lane) {
   const int i = s->word_seq[k];
   const int wi = static_cast<int>(cw0 + k - s->tab.w0[i]);
@@ -258,17 +263,18 @@ __device__ __forceinline__ void score_word(const Args& a, Smem* s, int k, long l
   const bool valid = c < s->tab.nc[i];
   const float bias = s->tab.bias[i];
   const int b = s->tab.b[i];
-  const uint8_t* rp = s->kbuf + k * WORD_SMEM + lane * ROW_STRIDE;
+  const uint8_t* rp = s->kbuf + k * a.lk * WORD_SMEM + lane * ROW_STRIDE;
   float acc[MAX_L][2];
 #pragma unroll
   for (int l = 0; l < MAX_L; ++l) acc[l][0] = acc[l][1] = 0.f;
 #pragma unroll 4
   for (int j = 0; j < D_I / 8; ++j) {
     float kf[8];
-    unpack8(*reinterpret_cast<const uint4*>(rp + 16 * j), kf);
+    if (!PER_LAYER) unpack8(*reinterpret_cast<const uint4*>(rp + 16 * j), kf);
 #pragma unroll
     for (int l = 0; l < MAX_L; ++l) {
       if (l < a.L) {
+        if (PER_LAYER) unpack8(*reinterpret_cast<const uint4*>(rp + l * WORD_SMEM + 16 * j), kf);
         const float4 qa = *reinterpret_cast<const float4*>(&s->qs[i][l][8 * j]);
         const float4 qb = *reinterpret_cast<const float4*>(&s->qs[i][l][8 * j + 4]);
         float& u = acc[l][j & 1];
@@ -427,7 +433,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
   if (warp == 0) {
     const long long NW = warp_total_words(a, lane);
     const long long W0 = (cta * NW) / G, W1 = ((cta + 1) * NW) / G;
-    if (W1 > W0) issue_chunk(a, s, W0, W1 < W0 + CHUNK_WORDS ? W1 : W0 + CHUNK_WORDS, lane);
+    const long long cap = CHUNK_WORDS / a.lk;   // words whose key rows fit in kbuf
+    if (W1 > W0) issue_chunk(a, s, W0, W1 < W0 + cap ? W1 : W0 + cap, lane);
     if (lane == 0) s->nw_total = NW;
   } else {
     const int RQ = a.L * D_I;
@@ -438,8 +445,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
   const long long W0 = (cta * NW) / G, W1 = ((cta + 1) * NW) / G;
 
   // ---- phase B: keep words, one warp per word
-  for (long long cw0 = W0; cw0 < W1; cw0 += CHUNK_WORDS) {
-    const long long cw1 = W1 < cw0 + CHUNK_WORDS ? W1 : cw0 + CHUNK_WORDS;
+  const long long ccap = CHUNK_WORDS / a.lk;
+  for (long long cw0 = W0; cw0 < W1; cw0 += ccap) {
+    const long long cw1 = W1 < cw0 + ccap ? W1 : cw0 + ccap;
     if (cw0 != W0) {
       __syncthreads();                          // every warp is done with kbuf
       if (warp == 0) issue_chunk(a, s, cw0, cw1, lane);
@@ -450,7 +458,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
     __syncthreads();
     if (s->abort) break;
     const int nwc = static_cast<int>(cw1 - cw0);
-    for (int k = warp; k < nwc; k += NWARPS) score_word(a, s, k, cw0, lane);
+    for (int k = warp; k < nwc; k += NWARPS) {
+      if (a.lk > 1)
+        score_word<true>(a, s, k, cw0, lane);
+      else
+        score_word<false>(a, s, k, cw0, lane);
+    }
   }
   grid_sync(a, s, 2);
 
@@ -538,14 +551,16 @@ extern "C" size_t lsa_index_workspace_size(int32_t B, int32_t L, int32_t d_i, in
   return index_ws_layout(B, L, max_cand).total;
 }
 
-extern "C" lsa_status lsa_index(const uint16_t* h, const uint16_t* w_q, const float* bias,
-                                const uint16_t* k_idx, const int64_t* kidx_off,
-                                const int32_t* n_cand, int32_t B, int32_t L, int32_t D,
-                                int32_t d_i, int32_t max_cand, int32_t* sel_ids, int32_t* sel_cnt,
-                                int32_t cap, float* logits, uint32_t* layer_mask, void* ws,
-                                size_t ws_bytes, int32_t* err, void* stream) {
+extern "C" lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const float* bias,
+                                   const uint16_t* k_idx, int64_t kidx_layer_stride,
+                                   const int64_t* kidx_off, const int32_t* n_cand, int32_t B,
+                                   int32_t L, int32_t D, int32_t d_i, int32_t max_cand,
+                                   int32_t* sel_ids, int32_t* sel_cnt, int32_t cap, float* logits,
+                                   uint32_t* layer_mask, void* ws, size_t ws_bytes, int32_t* err,
+                                   void* stream) {
   if (!h || !w_q || !bias || !k_idx || !kidx_off || !n_cand || !sel_cnt || !ws || !err)
     return LSA_ERR_INVALID_ARG;
+  if (kidx_layer_stride < 0) return LSA_ERR_INVALID_ARG;
   if (cap > 0 && !sel_ids) return LSA_ERR_INVALID_ARG;
   if (B <= 0 || B > 65535 || L < 1 || L > lsa::idx::MAX_L || d_i != lsa::idx::D_I || D <= 0 ||
       D % 256 != 0 || max_cand < 0 || cap < 0)
@@ -574,6 +589,8 @@ extern "C" lsa_status lsa_index(const uint16_t* h, const uint16_t* w_q, const fl
   a.w_q = w_q;
   a.bias = bias;
   a.k_idx = k_idx;
+  a.kls = kidx_layer_stride;
+  a.lk = kidx_layer_stride > 0 ? L : 1;
   a.kidx_off = kidx_off;
   a.n_cand = n_cand;
   a.q = reinterpret_cast<float*>(base + lay.q_off);
@@ -610,4 +627,14 @@ extern "C" lsa_status lsa_index(const uint16_t* h, const uint16_t* w_q, const fl
     return LSA_ERR_CUDA;
   }
   return LSA_OK;
+}
+
+extern "C" lsa_status lsa_index(const uint16_t* h, const uint16_t* w_q, const float* bias,
+                                const uint16_t* k_idx, const int64_t* kidx_off,
+                                const int32_t* n_cand, int32_t B, int32_t L, int32_t D,
+                                int32_t d_i, int32_t max_cand, int32_t* sel_ids, int32_t* sel_cnt,
+                                int32_t cap, float* logits, uint32_t* layer_mask, void* ws,
+                                size_t ws_bytes, int32_t* err, void* stream) {
+  return lsa_index_ex(h, w_q, bias, k_idx, 0, kidx_off, n_cand, B, L, D, d_i, max_cand, sel_ids,
+                      sel_cnt, cap, logits, layer_mask, ws, ws_bytes, err, stream);
 }

@@ -17,7 +17,8 @@ class LsaDecoder:
     """Owns the HBM pool, block tables, per-pass buffers and workspaces of a batch.
 
     w_q      bf16 [L][d_i][D]            (device)
-    k_idx    bf16 [rows][d_i]            (device); kidx_off int64 [B] row of block 0
+    k_idx    bf16 [rows][d_i] or [L][rows][d_i] per layer (device); kidx_off int64 [B]
+             row of block 0
     bias     f32 [B]
     host_pool bf16 [blocks][2][64][d]    pinned host cold pool; host_blk_off int64 [B+1]
     nb0      context blocks per sequence when pass 0 starts
@@ -78,6 +79,7 @@ class LsaDecoder:
         s.index_ws, s.index_ws_bytes = self.index_ws.data_ptr(), idx_bytes
         s.attn_ws, s.attn_ws_bytes = self.attn_ws.data_ptr(), attn_bytes
         s.err = self.err.data_ptr()
+        s.kidx_layer_stride = k_idx.shape[1] if k_idx.dim() == 3 else 0
         self.state = s
         _lib.check("lsa_state_check", _lib.lib().lsa_state_check(s))
 

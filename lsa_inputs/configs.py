@@ -33,6 +33,7 @@ class LsaConfig:
     ctx_uniform_blocks: Optional[tuple] = None  # (lo, hi) blocks, inclusive, drawn per sequence
     bias: Optional[List[float]] = None       # per-sequence indexer bias (shared by layers)
     bias_uniform: Optional[tuple] = None     # (lo, hi), drawn per sequence
+    kidx_per_layer: bool = False             # one compressed key table per indexer layer
     L: int = N_LAYERS
     d_i: int = D_INDEX
     block: int = BLOCK
@@ -78,6 +79,20 @@ def one_million(bias: float = -2.0) -> LsaConfig:
     return _fixed("1m_" + tag, 1, 1 << 20, 4096, 8192, 64, 512, bias, 1, 0)
 
 
+def one_million_layer_keys() -> LsaConfig:
+    """1M-token sequence at bias -2 whose three indexer layers each score against their
+    own compressed key table (K_idx [3][blocks][128])."""
+    c = _fixed("1m_b20_lk", 1, 1 << 20, 4096, 8192, 64, 512, -2.0, 1, 0)
+    c.kidx_per_layer = True
+    return c
+
+
+def one_million_latent() -> LsaConfig:
+    """1M-token sequence at bias -2 whose query encoders read a rank-2048 query latent
+    of the backbone instead of the 4096-wide hidden state (W_q [3][128][2048])."""
+    return _fixed("1m_b20_r2048", 1, 1 << 20, 2048, 8192, 64, 512, -2.0, 1, 0)
+
+
 def ragged_mix() -> LsaConfig:
     """B=64, context U{512..4096} blocks per sequence, bias U(-3,-1) per sequence, seed 7."""
     return LsaConfig(name="ragged_b64", B=64, D=4096, W=4096, H=64, d=512, passes=1, seed=7,
@@ -86,7 +101,7 @@ def ragged_mix() -> LsaConfig:
 
 def all_configs() -> List[LsaConfig]:
     return [tiny(), mid_batch(), long_ctx(), one_million(-1.5), one_million(-2.0),
-            one_million(-2.5), ragged_mix()]
+            one_million(-2.5), ragged_mix(), one_million_layer_keys(), one_million_latent()]
 
 
 def by_name(name: str) -> LsaConfig:

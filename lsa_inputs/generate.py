@@ -77,10 +77,18 @@ class Workload:
         self.total_blocks = int(off[-1])
 
         self.w_q = _randn_bf16((cfg.L, cfg.d_i, cfg.D), _gen(cfg.seed, "w_q"), cfg.wq_std)
-        self.k_idx = torch.empty((self.total_blocks, cfg.d_i), dtype=torch.bfloat16)
-        for b in range(B):
-            self.k_idx[off[b]:off[b + 1]] = _randn_bf16(
-                (int(self.nb_final[b]), cfg.d_i), _gen(cfg.seed, "k_idx", b))
+        if cfg.kidx_per_layer:
+            # one table per layer: [L][blocks][d_i]
+            self.k_idx = torch.empty((cfg.L, self.total_blocks, cfg.d_i), dtype=torch.bfloat16)
+            for l in range(cfg.L):
+                for b in range(B):
+                    self.k_idx[l, off[b]:off[b + 1]] = _randn_bf16(
+                        (int(self.nb_final[b]), cfg.d_i), _gen(cfg.seed, "k_idx_layer", l, b))
+        else:
+            self.k_idx = torch.empty((self.total_blocks, cfg.d_i), dtype=torch.bfloat16)
+            for b in range(B):
+                self.k_idx[off[b]:off[b + 1]] = _randn_bf16(
+                    (int(self.nb_final[b]), cfg.d_i), _gen(cfg.seed, "k_idx", b))
         self.host_pool = None
         if with_pool:
             self.host_pool = torch.empty((self.total_blocks, 2, blk, cfg.d), dtype=torch.bfloat16,
@@ -148,6 +156,9 @@ class Workload:
         return pages[:, 0].reshape(-1, d), pages[:, 1].reshape(-1, d)
 
     def seq_k_idx(self, b: int) -> torch.Tensor:
+        """Compressed keys of sequence b: [blocks][d_i], or [L][blocks][d_i] per layer."""
+        if self.k_idx.dim() == 3:
+            return self.k_idx[:, self.blk_off[b]:self.blk_off[b + 1]]
         return self.k_idx[self.blk_off[b]:self.blk_off[b + 1]]
 
 

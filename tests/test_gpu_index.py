@@ -19,7 +19,15 @@ CONFIGS = {
     "1m_b20": lambda: LI.one_million(-2.0),
     "1m_b25": lambda: LI.one_million(-2.5),
     "ragged_b64": LI.ragged_mix,
+    "1m_b20_lk": LI.one_million_layer_keys,
+    "1m_b20_r2048": LI.one_million_latent,
 }
+
+
+def cand_keys(wl, b, nc):
+    """bf16 bits of sequence b's first nc compressed keys ([nc][d_i] or [L][nc][d_i])."""
+    k = wl.seq_k_idx(b)
+    return bits(k[:, :nc] if k.dim() == 3 else k[:nc])
 
 
 def run_index(wl, p, cap=None, n_cand=None):
@@ -57,7 +65,7 @@ def test_index_matches_oracle(cuda_ok, name):
         n_near = 0
         for b in range(c.B):
             nc = n_cand[b]
-            ref_ids, z_ref = oracle.index_pass(bits(wl.w_q), hb[:, b], bits(wl.seq_k_idx(b)[:nc]),
+            ref_ids, z_ref = oracle.index_pass(bits(wl.w_q), hb[:, b], cand_keys(wl, b, nc),
                                                float(wl.bias[b]))
             dz = np.abs(z_gpu[:, b, :nc] - z_ref)
             assert dz.max(initial=0.0) <= LOGIT_ABS, (name, b, dz.max())

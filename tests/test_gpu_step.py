@@ -57,8 +57,9 @@ def check_loop(wl, keep_steps, heads=None):
         for b in range(c.B):
             n_ctx = int(wl.ctx_at(p)[b])
             nc = oracle.n_candidates(n_ctx, c.W)
-            ref_ids, z = oracle.index_pass(wq, hb[:, b], bits(wl.seq_k_idx(b)[:nc]),
-                                           float(wl.bias[b]))
+            kb = wl.seq_k_idx(b)
+            kb = kb[:, :nc] if kb.dim() == 3 else kb[:nc]
+            ref_ids, z = oracle.index_pass(wq, hb[:, b], bits(kb), float(wl.bias[b]))
             got = ids_gpu[b, :int(cnt_gpu[b])].tolist()
             near = compare_selection(got, ref_ids, z, "%s p%d b%d" % (c.name, p, b))
             # with near-tie flips, attention is checked over the GPU's own selection
@@ -88,6 +89,9 @@ STEPS = {0, 1, 31, 32, 33, 63}
     ("ragged_small", lambda: LI.scaled_down(LI.ragged_mix(), ctx_blocks=160, B=12)),
     ("one_million_geometry_small", lambda: LI.scaled_down(LI.one_million(-1.5), ctx_blocks=300)),
     ("window_covers_context", lambda: LI.scaled_down(LI.tiny(), ctx_blocks=12, W=1024)),
+    ("layer_keys_2pass_small", lambda: LI.scaled_down(LI.one_million_layer_keys(), ctx_blocks=300,
+                                                      passes=2)),
+    ("latent_input_small", lambda: LI.scaled_down(LI.one_million_latent(), ctx_blocks=300)),
 ])
 def test_scaled_loops(cuda_ok, name, cfg):
     wl = LI.Workload(cfg(), pin=True)
