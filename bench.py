@@ -186,16 +186,17 @@ class Inputs:
         self.v = torch.stack([b for _, b in kv]).to(dev)
 
 
-def make_decoder(wl, dev):
+def make_decoder(wl, dev, delta=False):
     import torch
     import lookahead_sparse_kv_lsa_b200 as lsa
     c = wl.cfg
     n_cand = [max(0, (int(x) - c.W) // c.block) for x in wl.ctx_at(0)]
-    max_cand = max(1, max(n_cand))
+    # room for the last pass's candidates (one more block per pass)
+    max_cand = max(1, max(max(0, (int(x) - c.W) // c.block) for x in wl.ctx_at(c.passes - 1)))
     dec = lsa.LsaDecoder(wl.w_q.to(dev), wl.k_idx.to(dev), wl.blk_off[:c.B],
                          torch.from_numpy(wl.bias).to(dev), wl.host_pool, wl.blk_off, wl.nb0,
                          W=c.W, H=c.H, cap=max_cand, max_cand=max_cand, scale=c.scale,
-                         sel_pages=min(c.B * max_cand, SEL_PAGES_CAP))
+                         sel_pages=min(c.B * max_cand, SEL_PAGES_CAP), delta_gather=delta)
     dec.load_window(0)
     return dec, n_cand
 
@@ -494,6 +495,39 @@ def e2e_measure(dec, wl, dev, passes, world):
             "ms_per_step": ms / passes, "api": "lsa_step (Python ctypes), pinned host buffers"}
 
 
+def delta_gather_report(wl, dev):
+    """Pass heads (set-up, indexer, gather) of every pass of a multi-pass workload, once
+    with the plain gather and once with resident-page reuse (lsa_gather_delta): gather
+    time and blocks copied over the host link. Decode steps are skipped, so the tail
+    pages written back hold no tokens; this runs after every other measurement."""
+    import torch
+    c = wl.cfg
+    res = {"passes": c.passes}
+    for mode in ("plain", "delta"):
+        dec, _ = make_decoder(wl, dev, delta=(mode == "delta"))
+        total_ms, kept = 0.0, 0
+        for p in range(c.passes):
+            h = wl.h(p).to(dev)
+            dec.pass_setup(p)
+            dec.index(h)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            dec.gather()
+            b.record()
+            torch.cuda.synchronize()
+            total_ms += a.elapsed_time(b)
+            kept += int(dec.sel_cnt.sum())
+        if dec.read_err() != 0:
+            raise SystemExit("device error word %d in the delta-gather report" % dec.read_err())
+        res[mode + "_gather_ms"] = total_ms
+        res["blocks_kept"] = kept
+        if mode == "delta":
+            res["blocks_copied"] = int(dec.copied.item())
+        del dec
+        torch.cuda.empty_cache()
+    return res
+
+
 def spot_check(wl, out, dec):
     """Compare the bench run's last decode step with the oracle on two heads."""
     import numpy as np
@@ -619,6 +653,8 @@ def run_lsa(args, rank, world, local):
         # the default workload samples all 64 steps; the others four of them
         steps = tuple(range(cfg.tau)) if cfg.name == DEFAULT_WORKLOAD else (0, 21, 42, 63)
         line["cpu_baseline"] = cpu_baseline(wl, steps)
+    if cfg.passes > 1:
+        line["delta_gather"] = delta_gather_report(wl, dev)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0

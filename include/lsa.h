@@ -152,6 +152,35 @@ lsa_status lsa_gather(const uint16_t* host_pool, int64_t host_blocks,
                       int32_t* err, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * lsa_gather_delta -- lsa_gather with resident-page reuse across passes (section 2 step 5,
+ * "refresh the loaded set"): a block kept by this pass and by the previous one keeps its
+ * HBM page and is not copied again; only blocks new to this pass cross the host link,
+ * into pages no kept block holds any more. The block table is built as by lsa_gather.
+ *
+ *   kept_ids, kept_pages  device i32 [B][cap]: the previous pass's kept blocks (ascending)
+ *                         and their pages; replaced by this pass's on return
+ *   kept_cnt              device i32 [B]: their number (0 at the start of a run; the
+ *                         step driver resets it at pass 0)
+ *   ws                    device workspace of lsa_gather_delta_workspace_size(B, cap,
+ *                         sel_page_count, n_sm) bytes, 16-byte aligned, zeroed before the
+ *                         first call (its barrier counters are left at zero)
+ *   copied                nullable device i32: incremented by the number of blocks copied
+ * Other arguments and errors as for lsa_gather. One cooperative launch (2 CTAs per SM)
+ * with three grid barriers; every wait is bounded.
+ */
+lsa_status lsa_gather_delta(const uint16_t* host_pool, int64_t host_blocks,
+                            const int64_t* host_blk_off, const int32_t* sel_ids,
+                            const int32_t* sel_cnt, int32_t cap, const int32_t* res_pages,
+                            const int32_t* n_res, int32_t res_stride, int32_t B, int32_t d,
+                            uint16_t* hbm_pool, int64_t n_pages, int32_t sel_page_base,
+                            int32_t sel_page_count, int32_t* block_table, int32_t bt_stride,
+                            int32_t* n_entries, int32_t* kept_ids, int32_t* kept_pages,
+                            int32_t* kept_cnt, void* ws, size_t ws_bytes, int32_t* copied,
+                            int32_t* err, void* stream);
+size_t lsa_gather_delta_workspace_size(int32_t B, int32_t cap, int32_t sel_page_count,
+                                       int32_t n_sm);
+
+/* ---------------------------------------------------------------------------------
  * lsa_decode_attn -- one decode step of block-sparse MQA attention (section 2 step 4):
  * every query head of sequence b attends to the tokens of the pages listed in its
  * block table, one KV head shared by all heads:
@@ -271,6 +300,12 @@ typedef struct lsa_state {
   int32_t* err;                        /* device i32 error word */
   int64_t kidx_layer_stride;           /* 0: K_idx shared by the layers; > 0: rows from
                                           layer l's key table to layer l+1's (lsa_index_ex) */
+  /* resident-page reuse across passes (lsa_gather_delta); all null: plain lsa_gather */
+  int32_t* kept_ids;                   /* device i32 [B][cap] */
+  int32_t* kept_pages;                 /* device i32 [B][cap] */
+  int32_t* kept_cnt;                   /* device i32 [B]; reset by lsa_pass_setup at pass 0 */
+  void* gather_ws; size_t gather_ws_bytes; /* lsa_gather_delta_workspace_size(B, cap,
+                                              n_pages - B*(W/64+1), n_sm), zeroed once */
 } lsa_state;
 
 /* Host-side validation of a state (no device work). */

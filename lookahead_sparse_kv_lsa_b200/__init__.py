@@ -14,7 +14,8 @@ import torch
 from . import _lib
 from ._lib import LsaError, LsaState, BLOCK, TAU
 
-__all__ = ["lsa_index", "lsa_gather", "lsa_decode_attn", "lsa_step", "lsa_load_window",
+__all__ = ["lsa_index", "lsa_gather", "lsa_gather_delta", "lsa_decode_attn", "lsa_step",
+           "lsa_load_window", "gather_delta_workspace_size",
            "lsa_pass_setup", "lsa_append", "lsa_decode_step",
            "index_workspace_size", "decode_attn_workspace_size", "LsaDecoder", "LsaError",
            "LsaState", "BLOCK", "TAU", "library_path"]
@@ -102,6 +103,35 @@ def lsa_gather(host_pool, host_blk_off, sel_ids, sel_cnt, res_pages, n_res, hbm_
         _dev(n_entries, torch.int32, "n_entries", B), _dev(err, torch.int32, "err", 1),
         _stream(stream))
     _lib.check("lsa_gather", st)
+
+
+def gather_delta_workspace_size(B: int, cap: int, sel_page_count: int,
+                                n_sm: Optional[int] = None) -> int:
+    if n_sm is None:
+        n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return int(_lib.lib().lsa_gather_delta_workspace_size(B, cap, sel_page_count, n_sm))
+
+
+def lsa_gather_delta(host_pool, host_blk_off, sel_ids, sel_cnt, res_pages, n_res, hbm_pool,
+                     sel_page_base: int, sel_page_count: int, block_table, n_entries, kept_ids,
+                     kept_pages, kept_cnt, ws, err, copied=None, stream=None) -> None:
+    """lsa_gather with resident-page reuse across passes (lsa_gather_delta in lsa.h)."""
+    if host_pool.is_cuda or not host_pool.is_pinned() or host_pool.dtype != torch.bfloat16:
+        raise ValueError("host_pool must be a pinned host bf16 tensor")
+    B = sel_cnt.shape[0]
+    d = hbm_pool.shape[-1]
+    cap = sel_ids.shape[1]
+    st = _lib.lib().lsa_gather_delta(
+        host_pool.data_ptr(), host_pool.shape[0], _dev(host_blk_off, torch.int64, "host_blk_off", B),
+        _dev(sel_ids, torch.int32, "sel_ids"), _dev(sel_cnt, torch.int32, "sel_cnt", B), cap,
+        _dev(res_pages, torch.int32, "res_pages"), _dev(n_res, torch.int32, "n_res", B),
+        res_pages.shape[1], B, d, _dev(hbm_pool, torch.bfloat16, "hbm_pool"), hbm_pool.shape[0],
+        sel_page_base, sel_page_count, _dev(block_table, torch.int32, "block_table"),
+        block_table.shape[1], _dev(n_entries, torch.int32, "n_entries", B),
+        _dev(kept_ids, torch.int32, "kept_ids", B * cap), _dev(kept_pages, torch.int32, "kept_pages", B * cap),
+        _dev(kept_cnt, torch.int32, "kept_cnt", B), _dev(ws, torch.uint8, "ws"), ws.numel(),
+        _opt(copied, torch.int32, "copied", 1), _dev(err, torch.int32, "err", 1), _stream(stream))
+    _lib.check("lsa_gather_delta", st)
 
 
 def lsa_decode_attn(q, hbm_pool, block_table, n_entries, tail_len, scale: float, out, ws, err,

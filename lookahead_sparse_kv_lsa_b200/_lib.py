@@ -44,6 +44,8 @@ class LsaState(C.Structure):
         ("attn_ws", _p), ("attn_ws_bytes", _sz),
         ("err", _p),
         ("kidx_layer_stride", _i64),
+        ("kept_ids", _p), ("kept_pages", _p), ("kept_cnt", _p),
+        ("gather_ws", _p), ("gather_ws_bytes", _sz),
     ]
 
 
@@ -58,6 +60,9 @@ SIGNATURES = {
     "lsa_index_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
     "lsa_gather": (_i32, [_p, _i64, _p, _p, _p, _i32, _p, _p, _i32, _i32, _i32, _p, _i64, _i32,
                           _i32, _p, _i32, _p, _p, _p]),
+    "lsa_gather_delta": (_i32, [_p, _i64, _p, _p, _p, _i32, _p, _p, _i32, _i32, _i32, _p, _i64,
+                                _i32, _i32, _p, _i32, _p, _p, _p, _p, _p, _sz, _p, _p, _p]),
+    "lsa_gather_delta_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
     "lsa_decode_attn": (_i32, [_p, _p, _i64, _p, _i32, _p, _p, _i32, _i32, _i32, C.c_float, _p,
                                _p, _sz, _p, _p]),
     "lsa_decode_attn_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),

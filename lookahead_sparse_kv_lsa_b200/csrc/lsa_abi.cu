@@ -95,6 +95,16 @@ extern "C" lsa_status lsa_state_check(const lsa_state* st) {
     return LSA_ERR_INVALID_ARG;
   if (st->index_ws_bytes < lsa_index_workspace_size(st->B, st->L, st->d_i, st->max_cand))
     return LSA_ERR_INVALID_ARG;
+  if (st->kidx_layer_stride < 0) return LSA_ERR_INVALID_ARG;
+  if (st->kept_cnt != nullptr) {               // resident-page reuse across passes
+    if (st->cap > 0 && (!st->kept_ids || !st->kept_pages)) return LSA_ERR_INVALID_ARG;
+    const int n_sm = lsa_host::sm_count();
+    const int64_t sel_pages = st->n_pages - static_cast<int64_t>(st->B) * wb1;
+    if (!st->gather_ws || n_sm <= 0 || sel_pages > INT32_MAX ||
+        st->gather_ws_bytes < lsa_gather_delta_workspace_size(st->B, st->cap,
+                                                              static_cast<int32_t>(sel_pages), n_sm))
+      return LSA_ERR_INVALID_ARG;
+  }
   return LSA_OK;
 }
 

@@ -28,7 +28,7 @@ class LsaDecoder:
 
     def __init__(self, w_q, k_idx, kidx_off, bias, host_pool, host_blk_off, nb0, W: int,
                  H: int, cap: int, max_cand: int, scale: float, sel_pages: Optional[int] = None,
-                 device=None):
+                 device=None, delta_gather: bool = False):
         dev = torch.device(device) if device is not None else w_q.device
         self.device = dev
         L, d_i, D = w_q.shape
@@ -80,6 +80,18 @@ class LsaDecoder:
         s.attn_ws, s.attn_ws_bytes = self.attn_ws.data_ptr(), attn_bytes
         s.err = self.err.data_ptr()
         s.kidx_layer_stride = k_idx.shape[1] if k_idx.dim() == 3 else 0
+        self.delta_gather = delta_gather
+        if delta_gather:     # resident-page reuse across passes
+            self.kept_ids = torch.zeros((B, max(1, cap)), **i32)
+            self.kept_pages = torch.zeros((B, max(1, cap)), **i32)
+            self.kept_cnt = torch.zeros(B, **i32)
+            self.copied = torch.zeros(1, **i32)
+            gbytes = _lib.lib().lsa_gather_delta_workspace_size(
+                B, cap, self.n_pages - B * wb1, n_sm)
+            self.gather_ws = torch.zeros(gbytes, dtype=torch.uint8, device=dev)
+            s.kept_ids, s.kept_pages = self.kept_ids.data_ptr(), self.kept_pages.data_ptr()
+            s.kept_cnt = self.kept_cnt.data_ptr()
+            s.gather_ws, s.gather_ws_bytes = self.gather_ws.data_ptr(), gbytes
         self.state = s
         _lib.check("lsa_state_check", _lib.lib().lsa_state_check(s))
 
@@ -103,8 +115,14 @@ class LsaDecoder:
                   self.index_ws, self.err, stream=stream)
 
     def gather(self, stream=None) -> None:
-        from . import lsa_gather
+        from . import lsa_gather, lsa_gather_delta
         base = self.B * (self.W // BLOCK + 1)
+        if self.delta_gather:
+            lsa_gather_delta(self.host_pool, self.host_blk_off, self.sel_ids, self.sel_cnt,
+                             self.res_pages, self.n_res, self.hbm_pool, base, self.n_pages - base,
+                             self.block_table, self.n_entries, self.kept_ids, self.kept_pages,
+                             self.kept_cnt, self.gather_ws, self.err, self.copied, stream)
+            return
         lsa_gather(self.host_pool, self.host_blk_off, self.sel_ids, self.sel_cnt, self.res_pages,
                    self.n_res, self.hbm_pool, base, self.n_pages - base, self.block_table,
                    self.n_entries, self.err, stream)
