@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", action="store_true",
+                    help="under torchrun: split the batch's sequences over the ranks "
+                         "(strong scaling of one workload) instead of one replica per GPU")
     return ap.parse_args()
 
 
@@ -437,6 +440,12 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
+def shard_range(B, rank, world):
+    """Sequences [lo, hi) of rank `rank` when B sequences are split over `world` ranks
+    (contiguous, sizes differing by at most one; every sequence in exactly one shard)."""
+    return (rank * B) // world, ((rank + 1) * B) // world
+
+
 def whole_job_rate(tokens_per_rank, world, max_ms):
     """Replicas: every rank decodes its own batch; the job rate is all ranks' tokens over
     the slowest rank's time."""
@@ -449,7 +458,7 @@ def barrier(world):
         dist.barrier()
 
 
-def e2e_measure(dec, wl, dev, passes, world):
+def e2e_measure(dec, wl, dev, passes, world, total_seqs=None):
     """Throughput through lsa_step from Python with host buffers: each decode step copies
     its inputs host->device (and h at the pass start) and reads its output back."""
     import torch
@@ -490,7 +499,8 @@ def e2e_measure(dec, wl, dev, passes, world):
     barrier(world)
     h2d = h_host.numel() * 2 + c.tau * (q_host[0].numel() + 2 * k_host[0].numel()) * 2
     d2h = c.tau * out_host[0].numel() * 2
-    return {"value": world * c.B * c.tau * passes / (ms * 1e-3), "unit": UNIT,
+    seqs = total_seqs if total_seqs is not None else world * c.B
+    return {"value": seqs * c.tau * passes / (ms * 1e-3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": ms / passes, "api": "lsa_step (Python ctypes), pinned host buffers"}
 
@@ -549,7 +559,16 @@ def run_lsa(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     cfg = LI.by_name(args.workload)
-    wl = LI.Workload(cfg, pin=True)
+    full_B = cfg.B
+    shard = args.shard and world > 1
+    if shard:
+        lo, hi = shard_range(cfg.B, rank, world)
+        if hi <= lo:
+            raise SystemExit("--shard needs at least one sequence per rank")
+        wl = LI.Workload(cfg, pin=True, seqs=range(lo, hi))
+    else:
+        wl = LI.Workload(cfg, pin=True)
+    cfg = wl.cfg
     dec, n_cand = make_decoder(wl, dev)
     inp = Inputs(wl, dev)
     out = torch.empty((cfg.tau, cfg.B, cfg.H, cfg.d), dtype=torch.bfloat16, device=dev)
@@ -607,14 +626,17 @@ def run_lsa(args, rank, world, local):
     h2d_peak = pinned_h2d_gbs(dev)
 
     line = {
-        "metric": METRIC, "value": whole_job_rate(cfg.B * cfg.tau * args.steps, world, ms),
+        "metric": METRIC,
+        "value": (full_B * cfg.tau * args.steps / (ms * 1e-3) if shard
+                  else whole_job_rate(cfg.B * cfg.tau * args.steps, world, ms)),
         "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": workload_desc(cfg),
+        "higher_is_better": True, "scaling": "strong" if shard else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(LI.by_name(args.workload)),
                    "step": "1 indexer pass + gather + 64 decode steps (B*64 tokens)",
-                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "parallelism": ("sequences sharded over %d GPUs" % world if shard else
+                                   "replicas" if world > 1 else "single GPU"),
                    "l2": "inputs larger than L2: each decode step streams %.0f MB of attended KV"
                          % (attn_bytes / 1e6),
                    "launch": "one CUDA graph per step"},
@@ -648,7 +670,8 @@ def run_lsa(args, rank, world, local):
                          "bytes_ratio_sparse_over_dense": attn_bytes / dbytes,
                          "time_ratio_sparse_over_dense": attn_avg_ms / dms}
     if not args.no_e2e:
-        line["e2e"] = e2e_measure(dec, wl, dev, args.steps, world)
+        line["e2e"] = e2e_measure(dec, wl, dev, args.steps, world,
+                                  total_seqs=full_B if shard else None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # the default workload samples all 64 steps; the others four of them
         steps = tuple(range(cfg.tau)) if cfg.name == DEFAULT_WORKLOAD else (0, 21, 42, 63)

@@ -16,10 +16,11 @@ simply history position N_p + s.
 """
 from __future__ import annotations
 
+import dataclasses
 import hashlib
 import os
 from concurrent.futures import ThreadPoolExecutor
-from typing import Optional
+from typing import Optional, Sequence
 
 import numpy as np
 import torch
@@ -49,7 +50,9 @@ class Workload:
     """All inputs of one LSA decode run (one config)."""
 
     def __init__(self, cfg: LsaConfig, pin: bool = False, threads: Optional[int] = None,
-                 with_pool: bool = True):
+                 with_pool: bool = True, seqs: Optional[Sequence[int]] = None):
+        """seqs: restrict the run to these sequences of the batch (a shard). Every tensor
+        holds exactly the values the whole-batch workload draws for those sequences."""
         self.cfg = cfg
         B, blk = cfg.B, cfg.block
         # context lengths (tokens at pass 0) and per-sequence bias
@@ -67,6 +70,19 @@ class Workload:
             g = _gen(cfg.seed, "bias")
             bias = (lo + (hi - lo) * torch.rand((B,), generator=g, dtype=torch.float64)).numpy()
             bias = bias.astype(np.float32)
+        # the whole batch's block offsets fix the cold pool's draws (chunks of blocks)
+        off_all = np.zeros(B + 1, dtype=np.int64)
+        off_all[1:] = np.cumsum(ctx // blk + cfg.passes)
+        self.seqs = np.arange(B) if seqs is None else np.asarray(list(seqs), dtype=np.int64)
+        if seqs is not None:
+            ctx, bias = ctx[self.seqs], bias[self.seqs]
+            self.cfg = cfg = dataclasses.replace(
+                cfg, name="%s_seqs%d-%d" % (cfg.name, int(self.seqs[0]), int(self.seqs[-1])),
+                B=len(self.seqs), ctx_tokens=[int(x) for x in ctx], ctx_uniform_blocks=None,
+                bias=[float(x) for x in bias], bias_uniform=None)
+            B = cfg.B
+        self._off_all = off_all
+        self._full_B = len(off_all) - 1
         self.ctx0 = ctx
         self.nb0 = ctx // blk
         self.nb_final = self.nb0 + cfg.passes
@@ -77,18 +93,19 @@ class Workload:
         self.total_blocks = int(off[-1])
 
         self.w_q = _randn_bf16((cfg.L, cfg.d_i, cfg.D), _gen(cfg.seed, "w_q"), cfg.wq_std)
+        gb = [int(x) for x in self.seqs]          # global sequence index of each row
         if cfg.kidx_per_layer:
             # one table per layer: [L][blocks][d_i]
             self.k_idx = torch.empty((cfg.L, self.total_blocks, cfg.d_i), dtype=torch.bfloat16)
             for l in range(cfg.L):
                 for b in range(B):
                     self.k_idx[l, off[b]:off[b + 1]] = _randn_bf16(
-                        (int(self.nb_final[b]), cfg.d_i), _gen(cfg.seed, "k_idx_layer", l, b))
+                        (int(self.nb_final[b]), cfg.d_i), _gen(cfg.seed, "k_idx_layer", l, gb[b]))
         else:
             self.k_idx = torch.empty((self.total_blocks, cfg.d_i), dtype=torch.bfloat16)
             for b in range(B):
                 self.k_idx[off[b]:off[b + 1]] = _randn_bf16(
-                    (int(self.nb_final[b]), cfg.d_i), _gen(cfg.seed, "k_idx", b))
+                    (int(self.nb_final[b]), cfg.d_i), _gen(cfg.seed, "k_idx", gb[b]))
         self.host_pool = None
         if with_pool:
             self.host_pool = torch.empty((self.total_blocks, 2, blk, cfg.d), dtype=torch.bfloat16,
@@ -99,14 +116,23 @@ class Workload:
     def _fill_pool(self, threads):
         n = self.total_blocks
         flat = self.host_pool.view(n, -1)
-        chunks = [(i, min(i + POOL_CHUNK_BLOCKS, n)) for i in range(0, n, POOL_CHUNK_BLOCKS)]
         seed = self.cfg.seed
+        n_all = int(self._off_all[-1])
+        # (global chunk, [global block range wanted], local destination of its first block)
+        chunks = []
+        for b, g in enumerate(int(x) for x in self.seqs):
+            g0, g1 = int(self._off_all[g]), int(self._off_all[g + 1])
+            c0 = (g0 // POOL_CHUNK_BLOCKS) * POOL_CHUNK_BLOCKS
+            for lo in range(c0, g1, POOL_CHUNK_BLOCKS):
+                hi = min(lo + POOL_CHUNK_BLOCKS, n_all)
+                a0, a1 = max(lo, g0), min(hi, g1)
+                chunks.append((lo, hi, a0, a1, int(self.blk_off[b]) + a0 - g0))
 
         def work(c):
-            lo, hi = c
+            lo, hi, a0, a1, dst = c
             x = torch.randn((hi - lo, flat.shape[1]), generator=_gen(seed, "pool", lo),
                             dtype=torch.float32)
-            flat[lo:hi].copy_(x)
+            flat[dst:dst + a1 - a0].copy_(x[a0 - lo:a1 - lo])
 
         nthr = threads or min(32, os.cpu_count() or 1)
         if len(chunks) == 1 or nthr == 1:
@@ -129,12 +155,14 @@ class Workload:
     def h(self, p: int) -> torch.Tensor:
         """Hidden states the indexer reads at the start of pass p: bf16 [L][B][D]."""
         c = self.cfg
-        return _randn_bf16((c.L, c.B, c.D), _gen(c.seed, "h", p))
+        x = _randn_bf16((c.L, self._full_B, c.D), _gen(c.seed, "h", p))
+        return x if c.B == self._full_B else x[:, torch.from_numpy(self.seqs)].contiguous()
 
     def q(self, p: int, s: int) -> torch.Tensor:
         """Queries of decode step s of pass p: bf16 [B][H][d]."""
         c = self.cfg
-        return _randn_bf16((c.B, c.H, c.d), _gen(c.seed, "q", p, s))
+        x = _randn_bf16((self._full_B, c.H, c.d), _gen(c.seed, "q", p, s))
+        return x if c.B == self._full_B else x[torch.from_numpy(self.seqs)].contiguous()
 
     def token_kv(self, b: int, pos: int):
         """(K, V) bf16 [d] of history position pos of sequence b."""

@@ -43,3 +43,24 @@ def test_distributions():
     assert abs(wq.std().item() * np.sqrt(4096) - 1.0) < 0.02
     pool = w.host_pool.float()
     assert abs(pool.mean().item()) < 0.01 and abs(pool.std().item() - 1.0) < 0.01
+
+
+def test_shard_holds_the_batch_draws():
+    """A workload restricted to some sequences holds exactly the whole batch's values for
+    them (the sequence-sharded multi-GPU run splits one workload, not a new one)."""
+    cfg = LI.scaled_down(LI.ragged_mix(), ctx_blocks=200, B=6)
+    full = LI.Workload(cfg)
+    part = LI.Workload(cfg, seqs=[2, 3, 4])
+    assert part.cfg.B == 3
+    for lb, gb in enumerate([2, 3, 4]):
+        assert torch.equal(part.seq_k_idx(lb), full.seq_k_idx(gb))
+        K1, V1 = part.seq_kv(lb)
+        K2, V2 = full.seq_kv(gb)
+        assert torch.equal(K1, K2) and torch.equal(V1, V2)
+        assert int(part.ctx0[lb]) == int(full.ctx0[gb])
+        assert float(part.bias[lb]) == float(full.bias[gb])
+    assert torch.equal(part.h(0), full.h(0)[:, 2:5])
+    assert torch.equal(part.q(0, 5), full.q(0, 5)[2:5])
+    k1, v1 = part.kv_new(0, 3)
+    k2, v2 = full.kv_new(0, 3)
+    assert torch.equal(k1, k2[2:5]) and torch.equal(v1, v2[2:5])

@@ -29,6 +29,12 @@ def _rank_main(rank, world, port, q):
         local_ms = 10.0 + 5.0 * rank            # rank 1 is the slow one
         ms = bench.max_over_ranks(local_ms, world)
         rate = bench.whole_job_rate(64 * 100, world, ms)
+        # sequence sharding of a 5-sequence batch: every sequence in exactly one shard
+        lo, hi = bench.shard_range(5, rank, world)
+        seqs = list(range(lo, hi))
+        gathered = [None] * world
+        dist.all_gather_object(gathered, seqs)
+        assert sorted(x for part in gathered for x in part) == list(range(5))
         q.put((rank, ms, rate))
     finally:
         dist.destroy_process_group()
