@@ -185,3 +185,39 @@ def decode_sequence(w_q_bits, k_idx_bits, K_bits, V_bits, bias: float, n_ctx0: i
                             block=block) for s in range(steps)]
         result.append((ids, z, outs))
     return result
+
+
+# ---------------------------------------------------------------------------------
+# Label denoising (training labels for the indexer)
+# ---------------------------------------------------------------------------------
+# "FlashMemory-DeepSeek-V4 Explained" (zhichai.net), section 3, "Label Denoising
+# Pipeline": the raw Lightning Indexer logits of each CSA layer are softmax-normalised
+# over the blocks; each layer keeps the smallest set of blocks whose cumulative
+# probability reaches p = 0.6 (top-p instead of a fixed top-k); a block is a positive
+# label of the token window when at least 3 of the 21 layers keep it.
+def softmax_f64(x: np.ndarray) -> np.ndarray:
+    """Softmax of one row in float64 (max-shifted)."""
+    x = np.asarray(x, dtype=np.float64)
+    e = np.exp(x - x.max())
+    return e / e.sum()
+
+
+def top_p_set(probs: np.ndarray, p: float) -> np.ndarray:
+    """Ids (ascending) of the smallest set of entries whose probabilities sum to >= p,
+    taking entries in decreasing probability, equal probabilities in increasing id."""
+    order = np.argsort(-probs, kind="stable")
+    cum = np.cumsum(probs[order])
+    k = int(np.searchsorted(cum, p, side="left"))    # first k with cum[k] >= p
+    k = min(k, len(order) - 1)
+    return np.sort(order[:k + 1])
+
+
+def denoise_labels(logits: np.ndarray, p: float = 0.6, min_votes: int = 3):
+    """logits float [n_layers][n_blocks] of one token window. Returns (labels, sets):
+    labels = ascending ids kept by at least min_votes layers; sets = each layer's
+    top-p set."""
+    sets = [top_p_set(softmax_f64(row), p) for row in logits]
+    votes = np.zeros(logits.shape[1], dtype=np.int64)
+    for s in sets:
+        votes[s] += 1
+    return np.flatnonzero(votes >= min_votes).astype(np.int64), sets

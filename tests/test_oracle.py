@@ -259,11 +259,64 @@ def check_per_layer_keys(O=O):
     assert np.allclose(same, O.block_logits(qr, kr, -2.0), rtol=1e-13, atol=1e-13)
 
 
+def check_top_p_closed_forms(O=O):
+    """Top-p on probabilities with known sums: exact boundary, ties by id, p = 1."""
+    pr = np.array([0.1, 0.4, 0.2, 0.3])          # sorted: 0.4 (1), 0.3 (3), 0.2 (2), 0.1 (0)
+    assert list(O.top_p_set(pr, 0.6)) == [1, 3]  # 0.4 + 0.3 = 0.7 >= 0.6
+    assert list(O.top_p_set(pr, 0.4)) == [1]     # reaches p exactly with one entry
+    assert list(O.top_p_set(pr, 0.71)) == [1, 2, 3]
+    assert list(O.top_p_set(pr, 1.0)) == [0, 1, 2, 3]
+    ties = np.full(8, 0.125)                     # equal probabilities: lower ids first
+    assert list(O.top_p_set(ties, 0.6)) == [0, 1, 2, 3, 4]
+    # softmax: uniform logits, and a closed form for two values
+    assert np.allclose(O.softmax_f64(np.zeros(5)), 0.2, rtol=0, atol=1e-15)
+    two = O.softmax_f64(np.array([math.log(3.0), 0.0]))
+    assert abs(two[0] - 0.75) < 1e-15 and abs(two[1] - 0.25) < 1e-15
+
+
+def check_top_p_bruteforce(O=O):
+    """Smallest subset reaching p, by exhaustive search over subsets on tiny rows."""
+    import itertools
+    rng = np.random.default_rng(8)
+    for trial in range(30):
+        n = int(rng.integers(1, 9))
+        pr = O.softmax_f64(rng.standard_normal(n) * 2.0)
+        p = float(rng.uniform(0.05, 0.95))
+        best = None
+        for k in range(1, n + 1):
+            for sub in itertools.combinations(range(n), k):
+                if pr[list(sub)].sum() >= p:
+                    best = k
+                    break
+            if best is not None:
+                break
+        got = O.top_p_set(pr, p)
+        assert len(got) == best
+        assert pr[got].sum() >= p
+        # it takes the largest probabilities
+        assert pr[got].min() >= np.sort(pr)[::-1][best - 1] - 1e-15
+
+
+def check_vote(O=O):
+    """Votes: a block is a label when at least 3 layers keep it."""
+    n = 6
+    logits = np.full((5, n), -50.0)
+    keep = {0: [0, 1], 1: [1, 2], 2: [1], 3: [2, 3], 4: [3, 5]}
+    for l, ids in keep.items():
+        logits[l, ids] = 10.0                    # one or two equal dominant entries
+    labels, sets = O.denoise_labels(logits, p=0.6, min_votes=3)
+    for l, ids in keep.items():
+        assert list(sets[l]) == ids              # two equal halves: both needed for 0.6
+    # votes: block 1 -> 3, blocks 2 and 3 -> 2, blocks 0 and 5 -> 1
+    assert list(labels) == [1]
+
+
 PINS = [check_bf16_decode, check_projection_unit_rows, check_projection_bruteforce,
         check_logits_closed_form, check_per_layer_keys, check_threshold_strict, check_union_bruteforce,
         check_selection_rate, check_single_token, check_two_token_closed_form,
         check_matches_sdpa, check_uniform_when_q_zero, check_attended_set,
-        check_special_cases_reduce_to_dense]
+        check_special_cases_reduce_to_dense, check_top_p_closed_forms, check_top_p_bruteforce,
+        check_vote]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -330,6 +383,15 @@ def _fails_some_pin(mutant):
     return False
 
 
+def _top_p_variant(pr, p, side="left", high_id=False, extra=0):
+    n = len(pr)
+    ids = np.arange(n)
+    order = np.lexsort((-ids if high_id else ids, -pr))
+    cum = np.cumsum(pr[order])
+    k = min(int(np.searchsorted(cum, p, side=side)) + extra, n - 1)
+    return np.sort(order[:k + 1])
+
+
 MUTANTS = {
     "logit_no_bias": dict(block_logits=lambda q, k, b: (q @ k.T) / math.sqrt(k.shape[1])),
     "logit_no_scale": dict(block_logits=lambda q, k, b: (q @ k.T) + b),
@@ -353,6 +415,10 @@ MUTANTS = {
         np.exp(sc * (q @ K.T)) @ V) / np.exp(sc * (q @ K.T)).sum(axis=1, keepdims=True) * 1.0001),
     "softmax_unscaled": dict(softmax_attention=lambda q, K, V, sc: O.softmax_attention(q, K, V, 1.0)),
     "candidates_include_window": dict(n_candidates=lambda n, W, block=64: n // block),
+    "top_p_strict_gt": dict(top_p_set=lambda pr, p: _top_p_variant(pr, p, side="right")),
+    "top_p_ties_by_high_id": dict(top_p_set=lambda pr, p: _top_p_variant(pr, p, high_id=True)),
+    "top_p_one_extra": dict(top_p_set=lambda pr, p: _top_p_variant(pr, p, extra=1)),
+    "vote_ge_2": dict(denoise_labels=lambda lg, p=0.6, min_votes=3: O.denoise_labels(lg, p, 2)),
     "bf16_truncated_wrong_shift": dict(bf16_to_f64=lambda b: (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(15)).view(np.float32).astype(np.float64)),
 }
 
