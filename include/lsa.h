@@ -53,6 +53,7 @@ typedef int32_t lsa_status;
 #define LSA_DEVERR_BAD_PAGE       4  /* a block-table entry or block id outside its pool; skipped */
 #define LSA_DEVERR_BAD_SIZE       8  /* a device-side count (n_cand, n_entries, tail_len) out of range */
 #define LSA_DEVERR_TIMEOUT       16  /* a bounded wait gave up */
+#define LSA_DEVERR_NUMERIC       32  /* a top-p search did not converge (non-finite logits) */
 
 #define LSA_BLOCK 64                 /* tokens per KV block / pool page */
 #define LSA_TAU   64                 /* decode steps per indexer pass */
@@ -339,6 +340,43 @@ lsa_status lsa_append(const lsa_state* st, int64_t step, const uint16_t* k_new,
    q: device bf16 [B][H][d]; k_new, v_new: device bf16 [B][d]; out: device bf16 [B][H][d]. */
 lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t* h, const uint16_t* q,
                     const uint16_t* k_new, const uint16_t* v_new, uint16_t* out, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * lsa_denoise_labels -- label denoising of the indexer's training targets (section 3
+ * "Label Denoising Pipeline", three steps): for each token window w and CSA layer l,
+ *
+ *   prob = softmax(logits[w][l][:])                       (step 1)
+ *   set[w][l] = the smallest set of blocks whose prob sums to >= top_p, taking blocks
+ *               by decreasing prob, equal probs by increasing block id   (step 2)
+ *   label[w][c] = 1 when block c is in set[w][l] for at least min_votes layers (step 3)
+ *
+ * The page's values are top_p = 0.6 and min_votes = 3 of 21 layers.
+ *
+ *   logits      device f32 [n_windows][n_layers][n_blocks], finite (a non-finite logit
+ *               gives unspecified sets and may set LSA_DEVERR_NUMERIC; nothing faults)
+ *   set_mask    device u32 [n_windows][n_layers][ceil(n_blocks/32)] out: bit (c % 32) of
+ *               word c / 32 is block c; bits past n_blocks are zero
+ *   set_cnt     nullable device i32 [n_windows][n_layers] out: the set sizes
+ *   label_mask  nullable device u32 [n_windows][ceil(n_blocks/32)] out
+ *   label_ids   device i32 [n_windows][label_cap] out: the labels in increasing id, the
+ *               first label_cap of them (may be null when label_cap == 0)
+ *   label_cnt   device i32 [n_windows] out: the number of labels (may exceed label_cap)
+ *   ws          device workspace of lsa_denoise_workspace_size(n_windows) bytes,
+ *               4-byte aligned, zeroed before the first call (per-window counters that
+ *               every call leaves at zero)
+ * Supported: 1 <= n_layers <= 63, 1 <= n_blocks <= LSA_DENOISE_MAX_BLOCKS,
+ * 0 < top_p <= 1; any min_votes (<= 0 keeps every block, > n_layers none).
+ * Ties in probability are ties in the fp32 logit, so the tie order is exact; where the
+ * running mass meets top_p within rounding (fp32 probabilities, fp64 sums) the boundary
+ * block may differ from an exact computation. One launch, one CTA per (window, layer).
+ */
+#define LSA_DENOISE_MAX_BLOCKS 45056
+lsa_status lsa_denoise_labels(const float* logits, int32_t n_windows, int32_t n_layers,
+                              int32_t n_blocks, double top_p, int32_t min_votes,
+                              uint32_t* set_mask, int32_t* set_cnt, uint32_t* label_mask,
+                              int32_t* label_ids, int32_t label_cap, int32_t* label_cnt,
+                              void* ws, size_t ws_bytes, int32_t* err, void* stream);
+size_t lsa_denoise_workspace_size(int32_t n_windows);
 
 #ifdef __cplusplus
 }

@@ -20,7 +20,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "liblsa_b200.so")
-SOURCES = ["lsa_abi.cu", "lsa_index.cu", "lsa_gather.cu", "lsa_attn.cu"]
+SOURCES = ["lsa_abi.cu", "lsa_index.cu", "lsa_gather.cu", "lsa_attn.cu", "lsa_denoise.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

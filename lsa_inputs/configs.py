@@ -127,3 +127,31 @@ def scaled_down(cfg: LsaConfig, ctx_blocks: int, B: Optional[int] = None,
     if cfg.bias is not None:
         out.bias = [cfg.bias[0]] * B
     return out
+
+
+
+@dataclasses.dataclass
+class DenoiseConfig:
+    """Synthetic Lightning-Indexer logits for the label-denoising workload: per token
+    window, `layers` CSA layers score `blocks` KV blocks. Logits are N(0, sigma^2) with
+    `relevant` blocks per window raised by `boost` in each layer with probability 1/2."""
+    name: str
+    windows: int
+    layers: int = 21
+    blocks: int = 16384
+    sigma: float = 1.0
+    boost: float = 5.0
+    relevant: int = 300
+    top_p: float = 0.6
+    min_votes: int = 3
+    seed: int = 0
+
+
+def denoise_1m() -> DenoiseConfig:
+    """64 token windows of a 1M-token context (16,384 blocks), 21 CSA layers."""
+    return DenoiseConfig(name="denoise_1m", windows=64)
+
+
+def denoise_tiny() -> DenoiseConfig:
+    """4 windows over 1,000 blocks (a row that is not a multiple of 32)."""
+    return DenoiseConfig(name="denoise_tiny", windows=4, blocks=1000, relevant=30, seed=3)

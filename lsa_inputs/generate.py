@@ -194,3 +194,21 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """The raw bf16 bit patterns of a tensor, as a numpy uint16 array (no conversion)."""
     assert t.dtype == torch.bfloat16
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def denoise_logits(cfg, w: int) -> torch.Tensor:
+    """Lightning-Indexer logits of token window w: float32 [layers][blocks]."""
+    x = torch.randn((cfg.layers, cfg.blocks), generator=_gen(cfg.seed, "dn_noise", w),
+                    dtype=torch.float32)
+    if cfg.sigma != 1.0:
+        x.mul_(cfg.sigma)
+    rel = torch.randperm(cfg.blocks, generator=_gen(cfg.seed, "dn_relevant", w))[:cfg.relevant]
+    active = torch.rand((cfg.layers, cfg.relevant), generator=_gen(cfg.seed, "dn_active", w)) < 0.5
+    for l in range(cfg.layers):
+        x[l, rel[active[l]]] += cfg.boost
+    return x
+
+
+def denoise_batch(cfg) -> torch.Tensor:
+    """All windows: float32 [windows][layers][blocks]."""
+    return torch.stack([denoise_logits(cfg, w) for w in range(cfg.windows)])
