@@ -9,40 +9,38 @@
 //   1. row max M, then e_i = 2^(x_i*log2(e) - M*log2(e)) for every block; a 16-bin
 //      histogram of the mass by whole logit units below M gives the total S and the bin
 //      j0 where the running mass from the top crosses T = top_p * S;
-//   2. one pass writes the mask words of the blocks above bin j0 (kept whatever the
-//      boundary) and appends the blocks of bin j0 to a candidate list, one segment per
-//      warp, without atomics;
-//   3. the list is split 16 ways, linearly in the order-preserving integer key of the
-//      logit, until at most 256 candidates remain; they are ranked by (logit descending,
-//      id ascending), their mass is scanned in that order in fp64, and the first rank
-//      whose running mass reaches T fixes the last kept (logit, id) pair. When all the
+//   2. one pass of warp ballots writes, per 32 blocks, the mask word of the blocks above
+//      bin j0 (kept whatever the boundary) and the word of the blocks in bin j0;
+//   3. the blocks of bin j0 become a candidate list in increasing id (one block-wide
+//      scan over the words); the list is split 16 ways, linearly in the
+//      order-preserving integer key of the logit, and narrowed in place, the entries
+//      above the chosen part OR-ed into the mask, until at most 256 candidates remain;
+//   4. those are ranked by (logit descending, id ascending), their mass is scanned in
+//      that order in fp64, and the first rank whose running mass reaches T fixes the
+//      last kept (logit, id); the kept candidates are OR-ed into the mask. When all the
 //      remaining candidates share one logit, the first m of them by id are kept, m the
-//      smallest count whose mass reaches T;
-//   4. the kept list entries are OR-ed into the mask words.
-// When bin j0 holds more blocks than the list, the bin itself is split over the row
-// first and the mask is then derived from the row. Ordering uses the exact fp32
-// logits, so blocks with equal probability are the blocks with equal logits and they
-// are taken by increasing id; only the position of the boundary depends on rounding
-// (fp32 e_i, fp64 sums).
+//      smallest count whose mass reaches T.
+// When bin j0 holds more blocks than the list, the bin is split the same way over the
+// row first. Ordering uses the exact fp32 logits, so blocks with equal probability are
+// the blocks with equal logits and they are taken by increasing id; only the position of
+// the boundary depends on rounding (fp32 e_i, fp64 sums).
 //
-// Each thread accumulates its share of a histogram in its own shared-memory column
-// (bank = lane), so no shared atomics are needed for the mass; the bins are then summed
-// in fp64. The vote runs in the last CTA of each window (a per-window ticket in the
-// workspace), as bit-sliced counters over the layers' 32-block mask words.
+// In the first pass each thread accumulates its share of the histogram in its own
+// shared-memory column (bank = lane), so the mass needs no shared atomics; the bins are
+// summed in fp64. The vote runs in the last CTA of each window (a per-window ticket in
+// the workspace), as bit-sliced counters over the layers' 32-block mask words.
 #include "lsa_common.cuh"
 
 namespace lsa {
 namespace {
 
-constexpr int NT = 256;               // threads per CTA
+constexpr int NT = 512;               // threads per CTA
 constexpr int NWARP = NT / 32;
 constexpr int DN_BINS = 16;
 constexpr int DN_CAND = 256;          // candidates resolved by ranking
 constexpr int DN_MAX_REFINE = 12;     // key-range splits; 9 always suffice for 32-bit keys
 constexpr int DN_PLANES = 6;          // vote counter bit planes: counts up to 63 layers
 constexpr int DN_LIST = 2048;         // candidate list
-constexpr int DN_SEG = DN_LIST / NWARP;  // one list segment per warp
-constexpr int DN_SLOTS = DN_LIST / NT;   // list slots per thread
 constexpr float DN_LOG2E = 1.4426950408889634f;
 
 struct DenoiseArgs {
@@ -60,37 +58,41 @@ struct DenoiseArgs {
   int32_t* err;
 };
 
-// Shared memory: this fixed part, then the row (NW * 32 floats), then NW mask words.
-struct Smem {
-  float hist[DN_BINS * NT];  // per-thread columns; later tie words
-  uint32_t lk[DN_LIST];      // candidate list keys, segment w at [w * DN_SEG, ...)
-  int32_t li[DN_LIST];       // and block ids
+// Shared memory: this fixed part, then the row (NW * 32 floats), the mask words (NW) and
+// the words of the blocks in the bin being resolved (NW). The first pass's per-thread
+// histogram columns and, after it, the candidate list share the area `u`.
+struct __align__(16) Smem {
+  float u[DN_BINS * NT];     // hist columns | list keys [DN_LIST], list ids [DN_LIST]
   double bsum[DN_BINS];
   double wsum[NWARP];
   double se[DN_CAND];        // candidate mass in rank order
-  uint32_t ckey[DN_CAND];    // candidates, in arrival order
-  int32_t cid[DN_CAND];
-  int32_t spos[DN_CAND];     // rank -> arrival slot
-  int32_t cw[NWARP];         // entries per list segment (more than DN_SEG: overflow)
+  int32_t spos[DN_CAND];     // rank -> list position
+  float lhist[NWARP][DN_BINS];  // list split: per-warp bin mass
   float wmax[NWARP];
   int32_t wcnt[NWARP];
-  int32_t c;                 // elements matched by the last compaction
-  uint32_t kmin, kmax;       // key range of those elements
+  uint32_t wkmin[NWARP], wkmax[NWARP];
+  int32_t c;                 // list entries
+  uint32_t kmin, kmax;       // their key range
   int32_t pick;              // rank of the last kept candidate
   uint32_t tau_key;          // the last kept (key, id)
   int32_t tau_id;
+  int32_t jsel;              // chosen bin (reduce_choose)
   int32_t last;              // this CTA closes its window
   int32_t total;
-  int32_t pad[3];
+  double acc;                // mass above the chosen bin
+  double total_mass;         // all bins' mass
+  double T;                  // top_p times the row's mass
 };
-static_assert(sizeof(Smem) % 16 == 0, "the row starts 16-byte aligned");
 
 extern __shared__ __align__(16) unsigned char dn_smem[];
 __device__ __forceinline__ Smem& sm() { return *reinterpret_cast<Smem*>(dn_smem); }
+__device__ __forceinline__ uint32_t* list_k() { return reinterpret_cast<uint32_t*>(sm().u); }
+__device__ __forceinline__ int32_t* list_i() { return reinterpret_cast<int32_t*>(sm().u) + DN_LIST; }
 __device__ __forceinline__ float* row_x() { return reinterpret_cast<float*>(dn_smem + sizeof(Smem)); }
-__device__ __forceinline__ uint32_t* row_words(int NW) {
+__device__ __forceinline__ uint32_t* mask_words(int NW) {
   return reinterpret_cast<uint32_t*>(row_x() + static_cast<size_t>(NW) * 32);
 }
+__device__ __forceinline__ uint32_t* bin_words(int NW) { return mask_words(NW) + NW; }
 
 // Order-preserving map of an fp32 value to uint32 (-0 taken as +0).
 __device__ __forceinline__ uint32_t order_key(float v) {
@@ -113,122 +115,140 @@ __device__ __forceinline__ float pow2(float y) {
 // Probability mass of one block up to the row's common factor 1/S.
 __device__ __forceinline__ float mass(float v, float ml2) { return pow2(fmaf(v, DN_LOG2E, -ml2)); }
 
-// Which elements a pass looks at: the first pass's unit bin jsel below the max, or a
-// key range [ka, kb] split into 16 linear key bins of which bin jsel is taken.
-struct Pred {
-  bool first;    // true: bin0(v) == jsel
-  float M;
-  uint32_t ka, kb;
-  uint64_t mul;  // floor(16 * 2^32 / (kb - ka + 1))
-  int jsel;      // -1: the whole key range
-};
-
 __device__ __forceinline__ int bin0(float v, float M) {
   return max(0, min(static_cast<int>(M - v), DN_BINS - 1));  // M - v >= 0 when finite
 }
-__device__ __forceinline__ int bin_key(uint32_t key, uint32_t kb, uint64_t mul) {
-  return static_cast<int>((static_cast<uint64_t>(kb - key) * mul) >> 32);
-}
-__device__ __forceinline__ bool pred_in(const Pred& p, float v, uint32_t key) {
-  if (p.first) return bin0(v, p.M) == p.jsel;
-  if (key < p.ka || key > p.kb) return false;
-  return p.jsel < 0 || bin_key(key, p.kb, p.mul) == p.jsel;
-}
-__device__ __forceinline__ Pred key_split(float M, uint32_t ka, uint32_t kb) {
+
+// 16 linear bins of the key range [ka, kb], bin 0 holding the largest keys.
+struct KeySplit {
+  uint32_t ka, kb;
+  uint64_t mul;  // floor(16 * 2^32 / (kb - ka + 1))
+};
+__device__ __forceinline__ KeySplit key_split(uint32_t ka, uint32_t kb) {
   const uint64_t R = static_cast<uint64_t>(kb - ka) + 1ull;
-  return Pred{false, M, ka, kb, (static_cast<uint64_t>(DN_BINS) << 32) / R, -1};
+  return KeySplit{ka, kb, (static_cast<uint64_t>(DN_BINS) << 32) / R};
+}
+__device__ __forceinline__ int bin_key(const KeySplit& k, uint32_t key) {
+  return static_cast<int>((static_cast<uint64_t>(k.kb - key) * k.mul) >> 32);
 }
 
-// Sum the NT per-thread histogram columns into s.bsum[] in fp64 (NT / 16 threads per bin).
-__device__ void reduce_bins() {
+// Block-wide exclusive scan of one int per thread; *total gets the sum, *klo / *khi the
+// min / max of the threads' key ranges lo / hi. Uses s.wcnt, s.wkmin, s.wkmax.
+__device__ __forceinline__ int block_scan(int v, int* total, uint32_t lo = 0xffffffffu,
+                                          uint32_t hi = 0u, uint32_t* klo = nullptr,
+                                          uint32_t* khi = nullptr) {
   Smem& s = sm();
-  constexpr int TPB = NT / DN_BINS;
-  const int tid = threadIdx.x;
-  const int b = tid / TPB, part = tid % TPB;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  __syncthreads();  // the previous use has been read
+  if (lane == 31) { s.wcnt[warp] = incl; s.wkmin[warp] = lo; s.wkmax[warp] = hi; }
+  __syncthreads();
+  int before = 0, all = 0;
+  uint32_t l = 0xffffffffu, h = 0u;
+#pragma unroll
+  for (int k = 0; k < NWARP; ++k) {
+    const int t = s.wcnt[k];
+    before += k < warp ? t : 0;
+    all += t;
+    l = min(l, s.wkmin[k]);
+    h = max(h, s.wkmax[k]);
+  }
+  *total = all;
+  if (klo) *klo = l;
+  if (khi) *khi = h;
+  return before + incl - v;
+}
+
+// Scans 16 bins in s.bsum from the top for the first non-empty bin where acc + the
+// running mass reaches T (the last non-empty bin when rounding leaves the total short
+// of T): s.jsel is that bin, s.acc the mass above it, s.total_mass the sum of all bins.
+// With top_p > 0, T is top_p times that sum (s.T). Warp 0 computes; every thread reads
+// the answer after the barrier.
+__device__ __forceinline__ void choose(double T, double acc, double top_p = 0.0) {
+  Smem& s = sm();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const double bj = lane < DN_BINS ? s.bsum[lane] : 0.0;
+    double incl = bj;  // running mass of bins 0..lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    const double total = __shfl_sync(0xffffffffu, incl, DN_BINS - 1);
+    if (top_p > 0.0) T = top_p * total;
+    const uint32_t nz = __ballot_sync(0xffffffffu, bj > 0.0);
+    const uint32_t hit = __ballot_sync(0xffffffffu, bj > 0.0 && acc + incl >= T);
+    const int j = hit ? __ffs(hit) - 1 : (nz ? 31 - __clz(nz) : 0);
+    const double above = __shfl_sync(0xffffffffu, incl - bj, j);
+    if (lane == 0) {
+      s.jsel = j;
+      s.acc = acc + above;
+      s.total_mass = total;
+      s.T = T;
+    }
+  }
+  __syncthreads();
+}
+
+// Sums the NT per-thread histogram columns into s.bsum (fp64; a warp per bin).
+__device__ __forceinline__ void reduce_columns() {
+  Smem& s = sm();
+  static_assert(NT / DN_BINS == 32, "one warp per bin");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   double v = 0.0;
 #pragma unroll 4
-  for (int k = 0; k < NT / TPB; ++k) v += s.hist[b * NT + part + TPB * k];
+  for (int k = 0; k < NT / 32; ++k) v += s.u[warp * NT + lane + 32 * k];
 #pragma unroll
-  for (int o = TPB / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if (part == 0) s.bsum[b] = v;
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) s.bsum[warp] = v;
   __syncthreads();
 }
 
-// Scanning the bins from the top, the first non-empty bin where acc + the running mass
-// reaches T (the last non-empty bin when rounding leaves the total short of T). acc
-// becomes the mass above the chosen bin. Every thread computes the same answer.
-__device__ int choose_bin(double T, double& acc) {
-  const double* bsum = sm().bsum;
-  double cum = acc, acc_last = acc;
-  int last_nz = -1;
-  for (int j = 0; j < DN_BINS; ++j) {
-    const double bj = bsum[j];
-    if (bj > 0.0) {
-      if (cum + bj >= T) { acc = cum; return j; }
-      last_nz = j;
-      acc_last = cum;
-    }
-    cum += bj;
-  }
-  acc = acc_last;
-  return last_nz < 0 ? 0 : last_nz;
-}
-
-// Warp-aggregated append of (key, id) for the lanes with `in` set; keeps s.c (all
-// matches), s.kmin / s.kmax; entries past `cap` are counted, not stored.
-__device__ __forceinline__ void append(bool in, uint32_t key, int id, uint32_t* ok, int32_t* oi,
-                                       int cap) {
-  Smem& s = sm();
-  const int lane = threadIdx.x & 31;
-  const uint32_t bal = __ballot_sync(0xffffffffu, in);
-  if (bal == 0u) return;
-  const int leader = __ffs(bal) - 1;
-  int slot0 = 0;
-  if (lane == leader) slot0 = atomicAdd(&s.c, __popc(bal));
-  slot0 = __shfl_sync(0xffffffffu, slot0, leader);
-  if (in) {
-    const int slot = slot0 + __popc(bal & ((1u << lane) - 1u));
-    if (slot < cap) { ok[slot] = key; oi[slot] = id; }
-    const uint32_t lo = __reduce_min_sync(bal, key), hi = __reduce_max_sync(bal, key);
-    if (lane == leader) { atomicMin(&s.kmin, lo); atomicMax(&s.kmax, hi); }
-  }
-}
-
-__device__ __forceinline__ void compact_begin() {
-  Smem& s = sm();
-  if (threadIdx.x == 0) { s.c = 0; s.kmin = 0xffffffffu; s.kmax = 0u; }
-  __syncthreads();
-}
-
-// ---------------------------------------------------------------- passes over the row
-// The row's blocks matched by p appended contiguously to the list (rare paths).
-__device__ __noinline__ void compact_row(int N, Pred p) {
+// The blocks marked in bin_words, in increasing id, into the list (the first DN_LIST of
+// them): s.c = their number, s.kmin / s.kmax their key range.
+__device__ __noinline__ void build_list(int NW) {
   Smem& s = sm();
   const float* x = row_x();
-  compact_begin();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int base = warp * 32; base < N; base += NT) {
-    const int i = base + lane;
-    float v = 0.f;
-    uint32_t key = 0u;
-    bool in = false;
-    if (i < N) { v = x[i]; key = order_key(v); in = pred_in(p, v, key); }
-    append(in, key, i, s.lk, s.li, DN_LIST);
-  }
-  __syncthreads();
-}
-
-__device__ __noinline__ void hist_row(int N, Pred p, float ml2) {
-  Smem& s = sm();
-  const float* x = row_x();
+  const uint32_t* bw = bin_words(NW);
   const int tid = threadIdx.x;
-#pragma unroll
-  for (int b = 0; b < DN_BINS; ++b) s.hist[b * NT + tid] = 0.f;
-  for (int i = tid; i < N; i += NT) {
-    const float v = x[i];
-    const uint32_t key = order_key(v);
-    if (key >= p.ka && key <= p.kb) s.hist[bin_key(key, p.kb, p.mul) * NT + tid] += mass(v, ml2);
+  const int per = (NW + NT - 1) / NT;
+  const int q0 = tid * per, q1 = min(NW, q0 + per);
+  int cnt = 0;
+  uint32_t lo = 0xffffffffu, hi = 0u;
+  for (int q = q0; q < q1; ++q) {
+    uint32_t b = bw[q];
+    cnt += __popc(b);
+    while (b != 0u) {
+      const uint32_t key = order_key(x[q * 32 + __ffs(b) - 1]);
+      b &= b - 1u;
+      lo = min(lo, key);
+      hi = max(hi, key);
+    }
   }
+  int total;
+  uint32_t klo, khi;
+  int pos = block_scan(cnt, &total, lo, hi, &klo, &khi);
+  uint32_t* lk = list_k();
+  int32_t* li = list_i();
+  for (int q = q0; q < q1 && pos < DN_LIST; ++q) {
+    uint32_t b = bw[q];
+    while (b != 0u && pos < DN_LIST) {
+      const int id = q * 32 + __ffs(b) - 1;
+      b &= b - 1u;
+      lk[pos] = order_key(x[id]);
+      li[pos] = id;
+      ++pos;
+    }
+  }
+  if (tid == 0) { s.c = total; s.kmin = klo; s.kmax = khi; }
   __syncthreads();
 }
 
@@ -241,24 +261,24 @@ __device__ __forceinline__ int tie_count(uint32_t tk, int c, double acc, double 
   return static_cast<int>(need);
 }
 
-// The last kept block is the m-th block of the row with key tk in id order.
-__device__ __noinline__ void tie_row(int N, int NW, uint32_t tk, int m) {
+// The id of the m-th (1-based) block marked in bin_words, in increasing id, into
+// s.tau_id (0x7fffffff when there are fewer).
+__device__ __noinline__ void mth_marked(int NW, int m) {
   Smem& s = sm();
-  const float* x = row_x();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t* words = reinterpret_cast<uint32_t*>(s.hist);  // NW <= DN_BINS * NT words
-  for (int q = warp; q < NW; q += NWARP) {
-    const int i = q * 32 + lane;
-    const uint32_t b = __ballot_sync(0xffffffffu, i < N && order_key(x[i]) == tk);
-    if (lane == 0) words[q] = b;
-  }
+  const uint32_t* bw = bin_words(NW);
+  const int tid = threadIdx.x;
+  const int per = (NW + NT - 1) / NT;
+  const int q0 = tid * per, q1 = min(NW, q0 + per);
+  int cnt = 0;
+  for (int q = q0; q < q1; ++q) cnt += __popc(bw[q]);
+  int total;
+  const int before = block_scan(cnt, &total);
+  if (tid == 0) s.tau_id = 0x7fffffff;
   __syncthreads();
-  if (tid == 0) {
-    s.tau_key = tk;
-    s.tau_id = 0x7fffffff;
-    int seen = 0;
-    for (int q = 0; q < NW; ++q) {
-      const uint32_t b = words[q];
+  if (m > before && m <= before + cnt) {
+    int seen = before;
+    for (int q = q0; q < q1; ++q) {
+      const uint32_t b = bw[q];
       const int n = __popc(b);
       if (seen + n >= m) {
         uint32_t bb = b;
@@ -269,102 +289,102 @@ __device__ __noinline__ void tie_row(int N, int NW, uint32_t tk, int m) {
       seen += n;
     }
   }
+  __syncthreads();
 }
 
-struct RowSplit {
-  double acc;
-  int done;
-};
-
-// Bin j0 holds more blocks than a list segment: compact it contiguously, and while it
-// exceeds the list split it by key, until its blocks fit (done = 0, the list holds them)
-// or share one logit (done = 1, tau fixed).
-__device__ __noinline__ RowSplit refine_row(const DenoiseArgs& a, float M, float ml2, double T,
-                                            double acc, int j0) {
+// Rare: bin j0 holds more than DN_LIST blocks. Split the marked blocks of the row by key
+// (the blocks above the chosen part join the mask words) until the marked part fits the
+// list or shares one logit. Returns 1 when tau is fixed (ties), 0 when the list holds
+// the part; acc is updated.
+__device__ __noinline__ int split_row(const DenoiseArgs& a, float ml2, double T, double* accp) {
   Smem& s = sm();
-  const int N = a.N;
-  compact_row(N, Pred{true, M, 0u, 0xffffffffu, 0ull, j0});
-  int c = s.c;
-  uint32_t kmin = s.kmin, kmax = s.kmax;
-  for (int it = 0; c > DN_LIST; ++it) {
+  const int N = a.N, NW = a.NW;
+  const float* x = row_x();
+  uint32_t* mw = mask_words(NW);
+  uint32_t* bw = bin_words(NW);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  double acc = *accp;
+  for (int it = 0;; ++it) {
+    const int c = s.c;
+    const uint32_t kmin = s.kmin, kmax = s.kmax;
+    if (c <= DN_LIST) { *accp = acc; return 0; }
     if (kmin == kmax) {
-      tie_row(N, a.NW, kmin, tie_count(kmin, c, acc, T, ml2));
-      return RowSplit{acc, 1};
+      mth_marked(NW, tie_count(kmin, c, acc, T, ml2));
+      if (tid == 0) s.tau_key = kmin;
+      __syncthreads();
+      *accp = acc;
+      return 1;
     }
     if (it == DN_MAX_REFINE) {  // unreachable: each split shrinks the key range 16-fold
-      if (threadIdx.x == 0) {
-        s.tau_key = kmax;
-        s.tau_id = 0x7fffffff;
-        set_err(a.err, LSA_DEVERR_NUMERIC);
-      }
-      return RowSplit{acc, 1};
+      if (tid == 0) { s.tau_key = kmax; s.tau_id = 0x7fffffff; set_err(a.err, LSA_DEVERR_NUMERIC); }
+      __syncthreads();
+      *accp = acc;
+      return 1;
     }
-    Pred q = key_split(M, kmin, kmax);
-    __syncthreads();  // every thread has read s.c, s.kmin, s.kmax and s.bsum
-    hist_row(N, q, ml2);
-    reduce_bins();
-    q.jsel = choose_bin(T, acc);
-    compact_row(N, q);
-    c = s.c;
-    kmin = s.kmin;
-    kmax = s.kmax;
-  }
-  return RowSplit{acc, 0};
-}
-
-// ---------------------------------------------------------------- the candidate list
-// Slot j = tid + NT*u (u < DN_SLOTS) of this thread is valid when bit u is set.
-__device__ __forceinline__ uint32_t list_slots() {
-  const Smem& s = sm();
-  uint32_t v = 0u;
+    const KeySplit ks = key_split(kmin, kmax);
+    float* col = s.u + tid;
+    __syncthreads();  // every thread has read s.c, s.kmin, s.kmax
 #pragma unroll
-  for (int u = 0; u < DN_SLOTS; ++u) {
-    const int j = threadIdx.x + NT * u;
-    if ((j % DN_SEG) < s.cw[j / DN_SEG]) v |= 1u << u;
-  }
-  return v;
-}
-
-// The list entries matched by p, into s.ckey / s.cid (s.c, s.kmin, s.kmax as for rows).
-__device__ __noinline__ void compact_list(uint32_t slots, Pred p) {
-  Smem& s = sm();
-  compact_begin();
-#pragma unroll
-  for (int u = 0; u < DN_SLOTS; ++u) {
-    const int j = threadIdx.x + NT * u;
-    uint32_t key = 0u;
-    int id = 0;
-    bool in = false;
-    if ((slots >> u) & 1u) {
-      key = s.lk[j];
-      id = s.li[j];
-      in = pred_in(p, key_value(key), key);
+    for (int b = 0; b < DN_BINS; ++b) col[b * NT] = 0.f;
+    for (int i = tid; i < N; i += NT) {
+      const uint32_t key = order_key(x[i]);
+      if (key >= kmin && key <= kmax) col[bin_key(ks, key) * NT] += mass(x[i], ml2);
     }
-    append(in, key, id, s.ckey, s.cid, DN_CAND);
+    __syncthreads();
+    reduce_columns();
+    choose(T, acc);
+    const int jsel = s.jsel;
+    acc = s.acc;
+    for (int q = warp; q < NW; q += NWARP) {
+      const int i = q * 32 + lane;
+      const uint32_t key = i < N ? order_key(x[i]) : 0u;
+      const bool in_range = i < N && key >= kmin && key <= kmax;
+      const int b = in_range ? bin_key(ks, key) : DN_BINS;
+      const uint32_t up = __ballot_sync(0xffffffffu, b < jsel);
+      const uint32_t in = __ballot_sync(0xffffffffu, b == jsel);
+      if (lane == 0) { mw[q] |= up; bw[q] = in; }
+    }
+    __syncthreads();
+    build_list(NW);
   }
-  __syncthreads();
 }
 
-__device__ __noinline__ void hist_list(uint32_t slots, Pred p, float ml2) {
-  Smem& s = sm();
-  float* col = s.hist + threadIdx.x;
-#pragma unroll
-  for (int b = 0; b < DN_BINS; ++b) col[b * NT] = 0.f;
-#pragma unroll
-  for (int u = 0; u < DN_SLOTS; ++u) {
-    if (!((slots >> u) & 1u)) continue;
-    const uint32_t key = s.lk[threadIdx.x + NT * u];
-    if (key >= p.ka && key <= p.kb) col[bin_key(key, p.kb, p.mul) * NT] += mass(key_value(key), ml2);
-  }
-  __syncthreads();
-}
-
-// Ranks candidates s.ckey/s.cid[0..c) (c >= 1) by (key desc, id asc), scans their mass
-// in rank order from acc and sets s.tau_key / s.tau_id to the first rank reaching T
-// (the last rank when none does).
+// Ranks the list's first c (1..DN_CAND) entries by (key desc, id asc), scans their mass
+// in rank order from acc and sets s.tau_key / s.tau_id to the first rank reaching T (the
+// last rank when none does).
 __device__ __noinline__ void rank_pick(int c, double acc, double T, float ml2) {
   Smem& s = sm();
+  const uint32_t* lk = list_k();
+  const int32_t* li = list_i();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (c <= 32) {  // one warp: lane j holds candidate j
+    if (warp == 0) {
+      const bool v = lane < c;
+      const uint32_t ki = v ? lk[lane] : 0u;
+      const int ii = v ? li[lane] : 0x7fffffff;
+      const double e = v ? static_cast<double>(mass(key_value(ki), ml2)) : 0.0;
+      int r = 0;
+      double before = 0.0;  // mass of the candidates ranked before this one
+      for (int j = 0; j < c; ++j) {
+        const uint32_t kj = __shfl_sync(0xffffffffu, ki, j);
+        const int ij = __shfl_sync(0xffffffffu, ii, j);
+        const bool ahead = (kj > ki) | ((kj == ki) & (ij < ii));
+        r += ahead;
+        const double ej = __shfl_sync(0xffffffffu, e, j);
+        if (ahead) before += ej;
+      }
+      const bool hit = v && acc + before + e >= T;
+      const int rmin = __reduce_min_sync(0xffffffffu, hit ? r : 0x7fffffff);
+      const int want = rmin == 0x7fffffff ? c - 1 : rmin;
+      const uint32_t who = __ballot_sync(0xffffffffu, v && r == want);
+      if (lane == __ffs(who) - 1) {
+        s.tau_key = ki;
+        s.tau_id = ii;
+      }
+    }
+    __syncthreads();
+    return;
+  }
   // G adjacent lanes share one candidate's comparisons (G a power of two, G * c <= NT)
   int G = 32;
   while (G > 1 && G * c > NT) G >>= 1;
@@ -372,11 +392,11 @@ __device__ __noinline__ void rank_pick(int c, double acc, double T, float ml2) {
   uint32_t ki = 0u;
   int ii = 0, r = 0;
   if (i < c) {
-    ki = s.ckey[i];
-    ii = s.cid[i];
+    ki = lk[i];
+    ii = li[i];
     for (int j = part; j < c; j += G) {
-      const uint32_t kj = s.ckey[j];
-      r += (kj > ki) | ((kj == ki) & (s.cid[j] < ii));
+      const uint32_t kj = lk[j];
+      r += (kj > ki) | ((kj == ki) & (li[j] < ii));
     }
   }
   for (int o = G / 2; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
@@ -400,49 +420,121 @@ __device__ __noinline__ void rank_pick(int c, double acc, double T, float ml2) {
   __syncthreads();
   if (tid == 0) {
     const int slot = s.spos[s.pick];
-    s.tau_key = s.ckey[slot];
-    s.tau_id = s.cid[slot];
+    s.tau_key = lk[slot];
+    s.tau_id = li[slot];
   }
+  __syncthreads();
 }
 
-// The list (every block of one bin of the row) narrowed by key splits to at most
-// DN_CAND candidates, which are ranked; fixes s.tau_key / s.tau_id.
-__device__ __noinline__ void resolve_list(const DenoiseArgs& a, float M, float ml2, double T,
-                                          double acc) {
+// The list (c entries in increasing id) narrowed to at most DN_CAND candidates and
+// resolved; the entries split off above the chosen part are OR-ed into the mask words.
+// Fixes s.tau_key / s.tau_id.
+__device__ __noinline__ void resolve_list(const DenoiseArgs& a, float ml2, double T, double acc) {
   Smem& s = sm();
-  const int tid = threadIdx.x;
-  const uint32_t slots = list_slots();
-  // all entries into the candidate arrays (when they fit), with their key range
-  Pred q{false, M, 0u, 0xffffffffu, 0ull, -1};
-  compact_list(slots, q);
-  int c = s.c;
-  uint32_t kmin = s.kmin, kmax = s.kmax;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t* lk = list_k();
+  int32_t* li = list_i();
+  uint32_t* mw = mask_words(a.NW);
   for (int it = 0;; ++it) {
+    const int c = s.c;
+    const uint32_t kmin = s.kmin, kmax = s.kmax;
     if (c == 0) {  // only for non-finite logits: the chosen bin always holds mass
       if (tid == 0) { s.tau_key = 0xffffffffu; s.tau_id = -1; set_err(a.err, LSA_DEVERR_NUMERIC); }
+      __syncthreads();
       return;
     }
     if (c <= DN_CAND) {
       rank_pick(c, acc, T, ml2);
       return;
     }
-    if (kmin == kmax) {  // every block of the row with this logit is in the list
-      tie_row(a.N, a.NW, kmin, tie_count(kmin, c, acc, T, ml2));
+    if (kmin == kmax) {  // all tied and in increasing id: the m-th entry is the last kept
+      if (tid == 0) {
+        s.tau_key = kmin;
+        s.tau_id = li[tie_count(kmin, c, acc, T, ml2) - 1];
+      }
+      __syncthreads();
       return;
     }
     if (it == DN_MAX_REFINE) {
       if (tid == 0) { s.tau_key = kmax; s.tau_id = 0x7fffffff; set_err(a.err, LSA_DEVERR_NUMERIC); }
+      __syncthreads();
       return;
     }
-    q = key_split(M, kmin, kmax);
-    __syncthreads();  // every thread has read s.c, s.kmin, s.kmax and s.bsum
-    hist_list(slots, q, ml2);
-    reduce_bins();
-    q.jsel = choose_bin(T, acc);
-    compact_list(slots, q);
-    c = s.c;
-    kmin = s.kmin;
-    kmax = s.kmax;
+    // split: per-warp bin mass by warp sums, one entry per thread per round
+    const KeySplit ks = key_split(kmin, kmax);
+    float part[DN_BINS];
+#pragma unroll
+    for (int b = 0; b < DN_BINS; ++b) part[b] = 0.f;
+    for (int j0 = 0; j0 < c; j0 += NT) {
+      const int j = j0 + tid;
+      int b = -1;
+      float e = 0.f;
+      if (j < c) {
+        const uint32_t key = lk[j];
+        b = bin_key(ks, key);
+        e = mass(key_value(key), ml2);
+      }
+#pragma unroll
+      for (int k = 0; k < DN_BINS; ++k) {
+        float t = b == k ? e : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        part[k] += t;
+      }
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int k = 0; k < DN_BINS; ++k) s.lhist[warp][k] = part[k];
+    }
+    __syncthreads();
+    if (tid < DN_BINS) {
+      double v = 0.0;
+      for (int w = 0; w < NWARP; ++w) v += s.lhist[w][tid];
+      s.bsum[tid] = v;
+    }
+    __syncwarp();  // bins 0..15 are warp 0's lanes: choose() reads them in warp 0 only
+    choose(T, acc);
+    const int jsel = s.jsel;
+    acc = s.acc;
+    // entries above the chosen part join the mask; the chosen part is kept, in order
+    uint32_t kk[DN_LIST / NT];
+    int32_t ki[DN_LIST / NT];
+    bool keep[DN_LIST / NT];
+#pragma unroll
+    for (int u = 0; u < DN_LIST / NT; ++u) {
+      const int j = u * NT + tid;  // round u holds entries [u * NT, (u + 1) * NT)
+      keep[u] = false;
+      kk[u] = 0u;
+      ki[u] = 0;
+      if (j < c) {
+        kk[u] = lk[j];
+        ki[u] = li[j];
+        const int b = bin_key(ks, kk[u]);
+        if (b < jsel) atomicOr(&mw[ki[u] >> 5], 1u << (ki[u] & 31));
+        keep[u] = b == jsel;
+      }
+    }
+    // order-preserving compaction in place: every read above precedes the first write
+    // (block_scan starts with a barrier); within a round the scan keeps thread order
+    int base = 0;
+    uint32_t klo = 0xffffffffu, khi = 0u;
+#pragma unroll
+    for (int u = 0; u < DN_LIST / NT; ++u) {
+      if (u * NT >= c) break;  // uniform
+      int tot_u;
+      uint32_t l, h;
+      const int pos = block_scan(keep[u] ? 1 : 0, &tot_u, keep[u] ? kk[u] : 0xffffffffu,
+                                 keep[u] ? kk[u] : 0u, &l, &h);
+      if (keep[u]) {
+        lk[base + pos] = kk[u];
+        li[base + pos] = ki[u];
+      }
+      base += tot_u;
+      klo = min(klo, l);
+      khi = max(khi, h);
+    }
+    if (tid == 0) { s.c = base; s.kmin = klo; s.kmax = khi; }
+    __syncthreads();
   }
 }
 
@@ -452,7 +544,7 @@ __device__ __noinline__ void resolve_list(const DenoiseArgs& a, float M, float m
 // scratch of NW words.
 __device__ __noinline__ void vote_window(const DenoiseArgs& a, int w, uint32_t* lab) {
   Smem& s = sm();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int NW = a.NW, L = a.L, vmin = a.min_votes;
   for (int q = tid; q < NW; q += NT) {
     uint32_t pl[DN_PLANES];
@@ -504,17 +596,8 @@ __device__ __noinline__ void vote_window(const DenoiseArgs& a, int w, uint32_t* 
   const int q0 = tid * per, q1 = min(NW, q0 + per);
   int cnt = 0;
   for (int q = q0; q < q1; ++q) cnt += __popc(lab[q]);
-  int incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
-  if (lane == 31) s.wcnt[warp] = incl;
-  __syncthreads();
-  int pos = incl - cnt;
-  for (int k = 0; k < warp; ++k) pos += s.wcnt[k];
-  if (tid == NT - 1) s.total = pos + cnt;
+  int total;
+  int pos = block_scan(cnt, &total);
   int32_t* ids = a.label_ids + static_cast<size_t>(w) * a.label_cap;
   for (int q = q0; q < q1 && pos < a.label_cap; ++q) {
     uint32_t b = lab[q];
@@ -523,11 +606,11 @@ __device__ __noinline__ void vote_window(const DenoiseArgs& a, int w, uint32_t* 
       b &= b - 1u;
     }
   }
-  __syncthreads();
   if (tid == 0) {
-    a.label_cnt[w] = s.total;
+    a.label_cnt[w] = total;
     a.tickets[w] = 0u;  // ready for the next call
   }
+  (void)s;
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -535,7 +618,8 @@ __global__ void __launch_bounds__(NT, 2) denoise_kernel(const __grid_constant__ 
   Smem& s = sm();
   const int N = a.N, NW = a.NW;
   float* x = row_x();
-  uint32_t* words = row_words(NW);
+  uint32_t* mw = mask_words(NW);
+  uint32_t* bw = bin_words(NW);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x;
   const int w = row / a.L;
@@ -571,7 +655,7 @@ __global__ void __launch_bounds__(NT, 2) denoise_kernel(const __grid_constant__ 
 
   // ---- pass 1: mass by whole units below the max
   {
-    float* col = s.hist + tid;
+    float* col = s.u + tid;
 #pragma unroll
     for (int b = 0; b < DN_BINS; ++b) col[b * NT] = 0.f;
 #pragma unroll 8
@@ -581,93 +665,65 @@ __global__ void __launch_bounds__(NT, 2) denoise_kernel(const __grid_constant__ 
     }
     __syncthreads();
   }
-  reduce_bins();
-  double S = 0.0;
-  for (int j = 0; j < DN_BINS; ++j) S += s.bsum[j];
-  const double T = a.top_p * S;
-  double acc = 0.0;
-  const int j0 = choose_bin(T, acc);
+  reduce_columns();
+  choose(0.0, 0.0, a.top_p);  // T = top_p * S with the row's total S
+  const double T = s.T;
+  double acc = s.acc;
+  const int j0 = s.jsel;
 
-  // ---- pass 2: mask words of the blocks above bin j0; bin j0 into the warp's segment
+  // ---- pass 2: per 32 blocks, the word of the blocks above bin j0 and of those in it.
+  // bin0(v) < j0  <=>  M - v < j0;  bin0(v) == j0  <=>  j0 <= M - v < j0 + 1 (any
+  // M - v from 15 on for the last bin), for finite logits.
   {
-    uint32_t* sk = s.lk + warp * DN_SEG;
-    int32_t* si = s.li + warp * DN_SEG;
-    int off = 0;
+    const float lo = static_cast<float>(j0), hi = static_cast<float>(j0 + 1);
+    const bool last_bin = j0 == DN_BINS - 1;
 #pragma unroll 4
     for (int q = warp; q < NW; q += NWARP) {
       const int i = q * 32 + lane;
-      const float v = i < N ? x[i] : -INFINITY;
-      const int jb = bin0(v, M);
-      const uint32_t ab = __ballot_sync(0xffffffffu, i < N && jb < j0);
-      if (lane == 0) words[q] = ab;
-      const bool in = i < N && jb == j0;
-      const uint32_t bb = __ballot_sync(0xffffffffu, in);
-      if (bb != 0u) {
-        if (in) {
-          const int slot = off + __popc(bb & ((1u << lane) - 1u));
-          if (slot < DN_SEG) { sk[slot] = order_key(v); si[slot] = i; }
-        }
-        off += __popc(bb);
-      }
-    }
-    if (lane == 0) s.cw[warp] = off;
-    __syncthreads();
-  }
-  bool ovf = false;
-#pragma unroll
-  for (int k = 0; k < NWARP; ++k) ovf |= s.cw[k] > DN_SEG;
-
-  // ---- rare: bin j0 overflowed a segment. Compact it contiguously (splitting it over
-  // the row while it exceeds the list); the mask is then derived from the row.
-  bool from_row = false;
-  int done = 0;
-  if (ovf) {
-    __syncthreads();  // every thread has read cw
-    const RowSplit rs = refine_row(a, M, ml2, T, acc, j0);
-    acc = rs.acc;
-    done = rs.done;
-    from_row = true;
-    __syncthreads();
-    if (tid < NWARP) {  // the contiguous list seen as segments
-      const int c = min(s.c, DN_LIST);
-      s.cw[tid] = max(0, min(DN_SEG, c - tid * DN_SEG));
+      const bool ok = i < N;
+      const float d = M - (ok ? x[i] : 0.f);
+      const uint32_t up = __ballot_sync(0xffffffffu, ok && d < lo);
+      const uint32_t in = __ballot_sync(0xffffffffu, ok && d >= lo && (last_bin || d < hi));
+      if (lane == 0) { mw[q] = up; bw[q] = in; }
     }
     __syncthreads();
   }
-  if (!done) resolve_list(a, M, ml2, T, acc);
-  __syncthreads();
 
+  // ---- the bin's blocks as a list (split over the row first when they overflow it)
+  build_list(NW);
+  int fixed = 0;
+  if (s.c > DN_LIST) fixed = split_row(a, ml2, T, &acc);
+  if (!fixed) resolve_list(a, ml2, T, acc);
+
+  // ---- the kept candidates into the mask words
   const uint32_t tk = s.tau_key;
   const int ti = s.tau_id;
-  if (!from_row) {
-    // ---- the kept list entries OR-ed into the words of the blocks above the bin
-    const uint32_t slots = list_slots();
-#pragma unroll
-    for (int u = 0; u < DN_SLOTS; ++u) {
-      if (!((slots >> u) & 1u)) continue;
-      const int j = tid + NT * u;
-      const uint32_t key = s.lk[j];
-      const int id = s.li[j];
-      if (key > tk || (key == tk && id <= ti)) atomicOr(&words[id >> 5], 1u << (id & 31));
-    }
-  } else {
-    // ---- the mask from the row
-    for (int q = warp; q < NW; q += NWARP) {
-      const int i = q * 32 + lane;
-      bool sel = false;
-      if (i < N) {
-        const uint32_t key = order_key(x[i]);
-        sel = key > tk || (key == tk && i <= ti);
+  {
+    const int c = min(s.c, DN_LIST);
+    const uint32_t* lk = list_k();
+    const int32_t* li = list_i();
+    if (!fixed) {
+      for (int j = tid; j < c; j += NT) {
+        const uint32_t key = lk[j];
+        const int id = li[j];
+        if (key > tk || (key == tk && id <= ti)) atomicOr(&mw[id >> 5], 1u << (id & 31));
       }
-      const uint32_t b = __ballot_sync(0xffffffffu, sel);
-      if (lane == 0) words[q] = b;
+    } else {
+      // ties over the row: the marked blocks with id up to tau_id
+      for (int q = tid; q < NW; q += NT) {
+        const int first = q * 32;
+        uint32_t b = bw[q];
+        if (first > ti) b = 0u;
+        else if (first + 31 > ti) b &= (2u << (ti - first)) - 1u;
+        mw[q] |= b;
+      }
     }
+    __syncthreads();
   }
-  __syncthreads();
   int cnt = 0;
   uint32_t* out = a.set_mask + static_cast<size_t>(row) * NW;
   for (int q = tid; q < NW; q += NT) {
-    const uint32_t b = words[q];
+    const uint32_t b = mw[q];
     out[q] = b;
     cnt += __popc(b);
   }
@@ -676,30 +732,32 @@ __global__ void __launch_bounds__(NT, 2) denoise_kernel(const __grid_constant__ 
 
   // ---- the row's set size, the window ticket, the vote when this row closes the window
   if (lane == 0) s.wcnt[warp] = cnt;
-  __threadfence();  // the mask words before the window's ticket
   __syncthreads();
   if (tid == 0) {
     int t = 0;
     for (int k = 0; k < NWARP; ++k) t += s.wcnt[k];
     if (a.set_cnt) a.set_cnt[row] = t;
+    // the CTA's mask stores, ordered before this thread by the barrier, become visible
+    // device-wide before the ticket (fence cumulativity)
     __threadfence();
     s.last = atomicAdd(&a.tickets[w], 1u) == static_cast<uint32_t>(a.L - 1);
   }
   __syncthreads();
   if (!s.last) return;
   __threadfence();
-  vote_window(a, w, words);
+  vote_window(a, w, bw);  // the bin words are scratch now
 }
 
 size_t smem_bytes(int32_t NW) {
   return sizeof(Smem) + static_cast<size_t>(NW) * 32 * sizeof(float) +
-         static_cast<size_t>(NW) * sizeof(uint32_t);
+         2 * static_cast<size_t>(NW) * sizeof(uint32_t);
 }
 
+static_assert(sizeof(Smem) % 16 == 0, "the row starts 16-byte aligned");
+static_assert(2 * DN_LIST * 4 <= sizeof(float) * DN_BINS * NT, "the list fits the shared area");
 static_assert(LSA_DENOISE_MAX_BLOCKS % 32 == 0, "whole mask words");
-static_assert(sizeof(Smem) + LSA_DENOISE_MAX_BLOCKS * 4 + LSA_DENOISE_MAX_BLOCKS / 8 <= 227 * 1024,
+static_assert(sizeof(Smem) + LSA_DENOISE_MAX_BLOCKS * 4 + LSA_DENOISE_MAX_BLOCKS / 4 <= 227 * 1024,
               "the longest row fits one CTA's shared memory");
-static_assert(LSA_DENOISE_MAX_BLOCKS / 32 <= DN_BINS * NT, "tie words fit the histogram area");
 static_assert(DN_CAND <= NT, "one scan lane per ranked candidate");
 
 }  // namespace
