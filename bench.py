@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-denoise", action="store_true",
+                    help="skip the label-denoising report (64 windows x 21 layers x 16,384 blocks)")
     ap.add_argument("--shard", action="store_true",
                     help="under torchrun: split the batch's sequences over the ranks "
                          "(strong scaling of one workload) instead of one replica per GPU")
@@ -538,6 +540,73 @@ def delta_gather_report(wl, dev):
     return res
 
 
+def denoise_report(dev, hbm, with_oracle=True, reps=20):
+    """Label denoising (lsa_denoise_labels) on 64 token windows x 21 CSA layers x 16,384
+    blocks of synthetic Lightning-Indexer logits: device time per launch over three
+    rotating copies of the logits (264 MB, larger than L2), the fraction of the HBM
+    bandwidth for the bytes the launch must move, and the oracle on two windows."""
+    import numpy as np
+    import torch
+    import lookahead_sparse_kv_lsa_b200 as lsa
+    import lsa_inputs as LI
+    cfg = LI.denoise_1m()
+    x = LI.denoise_batch(cfg)
+    W, L, N = x.shape
+    NW = (N + 31) // 32
+    cap = 4096
+    copies = [x.to(dev) for _ in range(3)]
+    set_mask = torch.empty((W, L, NW), dtype=torch.int32, device=dev)
+    set_cnt = torch.empty((W, L), dtype=torch.int32, device=dev)
+    label_mask = torch.empty((W, NW), dtype=torch.int32, device=dev)
+    label_ids = torch.empty((W, cap), dtype=torch.int32, device=dev)
+    label_cnt = torch.empty((W,), dtype=torch.int32, device=dev)
+    ws = torch.zeros(lsa.denoise_workspace_size(W), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def launch(i):
+        lsa.lsa_denoise_labels(copies[i % 3], set_mask, label_cnt, ws, err, top_p=cfg.top_p,
+                               min_votes=cfg.min_votes, set_cnt=set_cnt,
+                               label_mask=label_mask, label_ids=label_ids)
+    for i in range(3):
+        launch(i)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for i, (a, b) in enumerate(evs):
+        a.record()
+        launch(i)
+        b.record()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise SystemExit("device error word %d in the denoise report" % int(err.item()))
+    ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    counts = label_cnt.cpu().numpy()
+    nbytes = W * L * N * 4 + W * L * NW * 4 + W * NW * 4 + int(counts.sum()) * 4
+    res = {"workload": "64 windows x 21 layers x 16,384 blocks (fp32 logits, top_p 0.6, >= 3 votes)",
+           "ms": ms, "windows_per_s": W / (ms * 1e-3), "algorithmic_bytes": nbytes,
+           "achieved_GBs": nbytes / (ms * 1e-3) / 1e9, "frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
+           "mean_set_size": float(set_cnt.float().mean()), "mean_labels": float(counts.mean()),
+           "timing": "median of %d launches over 3 rotating input copies (264 MB)" % reps}
+    if with_oracle:
+        import oracle
+        lab = label_mask.cpu().numpy().view(np.uint32)
+        t0 = time.perf_counter()
+        diff = 0
+        for w in (0, W - 1):
+            o_labels, _ = oracle.denoise_labels(x[w].numpy(), p=cfg.top_p, min_votes=cfg.min_votes)
+            bits = np.unpackbits(lab[w].view(np.uint8), bitorder="little")[:N].astype(bool)
+            o = np.zeros(N, dtype=bool)
+            o[o_labels] = True
+            diff += int((bits != o).sum())
+        dt = time.perf_counter() - t0
+        res["oracle_label_mismatches_2_windows"] = diff
+        res["cpu_baseline"] = {"value": 2 / dt, "unit": "windows/s", "cores": oracle_threads(),
+                               "kind": "oracle", "sample": "windows 0 and 63 (2 x 21 rows)"}
+    del copies
+    torch.cuda.empty_cache()
+    return res
+
+
 def spot_check(wl, out, dec):
     """Compare the bench run's last decode step with the oracle on two heads."""
     import numpy as np
@@ -678,6 +747,8 @@ def run_lsa(args, rank, world, local):
         line["cpu_baseline"] = cpu_baseline(wl, steps)
     if cfg.passes > 1:
         line["delta_gather"] = delta_gather_report(wl, dev)
+    if rank == 0 and world == 1 and not args.no_denoise:
+        line["denoise"] = denoise_report(dev, hbm, with_oracle=not args.no_cpu_baseline)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
