@@ -76,7 +76,7 @@ struct __align__(16) Smem {
   int32_t pick;              // rank of the last kept candidate
   uint32_t tau_key;          // the last kept (key, id)
   int32_t tau_id;
-  int32_t jsel;              // chosen bin (reduce_choose)
+  int32_t jsel;              // chosen bin (choose)
   int32_t last;              // this CTA closes its window
   int32_t total;
   double acc;                // mass above the chosen bin
