@@ -342,6 +342,17 @@ lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t* h, const 
                     const uint16_t* k_new, const uint16_t* v_new, uint16_t* out, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * lsa_wait_selftest -- the library's bounded device wait, on its own: one thread polls
+ * *flag (device u32, acquire at gpu scope) until it is >= target, the same wait every
+ * grid barrier of the library uses. When limit_ns (1 .. 10^10) passes first, it ORs
+ * LSA_DEVERR_TIMEOUT into the device word *err and returns, so a caller can make the
+ * wait run out on a flag that nothing sets and check that the status arrives and the
+ * context stays usable. (The library's own barriers wait at most 2 s.)
+ */
+lsa_status lsa_wait_selftest(const uint32_t* flag, uint32_t target, int64_t limit_ns,
+                             int32_t* err, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * lsa_denoise_labels -- label denoising of the indexer's training targets (section 3
  * "Label Denoising Pipeline", three steps): for each token window w and CSA layer l,
  *

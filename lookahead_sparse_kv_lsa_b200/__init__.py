@@ -16,7 +16,7 @@ from ._lib import LsaError, LsaState, BLOCK, TAU
 
 __all__ = ["lsa_index", "lsa_gather", "lsa_gather_delta", "lsa_decode_attn", "lsa_step",
            "lsa_load_window", "gather_delta_workspace_size", "lsa_denoise_labels",
-           "denoise_workspace_size", "DENOISE_MAX_BLOCKS",
+           "denoise_workspace_size", "DENOISE_MAX_BLOCKS", "lsa_wait_selftest",
            "lsa_pass_setup", "lsa_append", "lsa_decode_step",
            "index_workspace_size", "decode_attn_workspace_size", "LsaDecoder", "LsaError",
            "LsaState", "BLOCK", "TAU", "library_path"]
@@ -160,6 +160,16 @@ def lsa_denoise_labels(logits, set_mask, label_cnt, ws, err, top_p: float = 0.6,
         _dev(label_cnt, torch.int32, "label_cnt", W), _dev(ws, torch.uint8, "ws"), ws.numel(),
         _dev(err, torch.int32, "err", 1), _stream(stream))
     _lib.check("lsa_denoise_labels", st)
+
+
+def lsa_wait_selftest(flag, target: int, limit_ns: int, err, stream=None) -> None:
+    """The library's bounded device wait on its own (lsa_wait_selftest in lsa.h): polls the
+    device u32 `flag` (an int32 tensor) until it reaches `target`, or ORs the timeout bit
+    into `err` after `limit_ns`."""
+    st = _lib.lib().lsa_wait_selftest(_dev(flag, torch.int32, "flag", 1), int(target) & 0xffffffff,
+                                      int(limit_ns), _dev(err, torch.int32, "err", 1),
+                                      _stream(stream))
+    _lib.check("lsa_wait_selftest", st)
 
 
 def lsa_decode_attn(q, hbm_pool, block_table, n_entries, tail_len, scale: float, out, ws, err,

@@ -19,6 +19,7 @@ DEVERR_POOL_CAPACITY = 2
 DEVERR_BAD_PAGE = 4
 DEVERR_BAD_SIZE = 8
 DEVERR_TIMEOUT = 16
+DEVERR_NUMERIC = 32
 
 BLOCK = 64
 TAU = 64
@@ -78,6 +79,7 @@ SIGNATURES = {
     "lsa_denoise_labels": (_i32, [_p, _i32, _i32, _i32, C.c_double, _i32, _p, _p, _p, _p, _i32,
                                   _p, _p, _sz, _p, _p]),
     "lsa_denoise_workspace_size": (_sz, [_i32]),
+    "lsa_wait_selftest": (_i32, [_p, C.c_uint32, _i64, _p, _p]),
 }
 
 _lib = None

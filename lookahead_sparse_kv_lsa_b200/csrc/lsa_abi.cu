@@ -75,6 +75,23 @@ extern "C" const char* lsa_status_str(lsa_status s) {
 
 extern "C" int32_t lsa_version(void) { return 100; }
 
+namespace {
+__global__ void wait_selftest_kernel(const unsigned int* flag, unsigned int target,
+                                     uint64_t limit_ns, int32_t* err) {
+  if (threadIdx.x == 0 && !lsa::spin_until_geq(flag, target, limit_ns))
+    lsa::set_err(err, LSA_DEVERR_TIMEOUT);
+}
+}  // namespace
+
+extern "C" lsa_status lsa_wait_selftest(const uint32_t* flag, uint32_t target, int64_t limit_ns,
+                                        int32_t* err, void* stream) {
+  if (flag == nullptr || err == nullptr || limit_ns < 1 || limit_ns > 10000000000LL)
+    return LSA_ERR_INVALID_ARG;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      flag, target, static_cast<uint64_t>(limit_ns), err);
+  return cudaPeekAtLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+}
+
 extern "C" lsa_status lsa_state_check(const lsa_state* st) {
   if (!st) return LSA_ERR_INVALID_ARG;
   if (st->B <= 0 || st->L < 1 || st->L > 4 || st->d_i != 128 || st->D <= 0 || st->D % 256 != 0)

@@ -367,16 +367,9 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
   if (tid == 0) {
     __threadfence();
     const unsigned int before = atomicAdd(a.sync, 1u);
-    const uint64_t t0 = globaltimer_ns();
-    bool ok = true;
-    while (before + 1u < static_cast<unsigned int>(G) &&
-           ld_acquire_gpu(a.sync) < static_cast<unsigned int>(G)) {
-      __nanosleep(32);
-      if (globaltimer_ns() - t0 > LSA_WAIT_LIMIT_NS) {
-        ok = false;
-        break;
-      }
-    }
+    // the last CTA to arrive does not wait
+    const bool ok = before + 1u >= static_cast<unsigned int>(G) ||
+                    spin_until_geq(a.sync, static_cast<unsigned int>(G));
     __threadfence();
     fence_proxy_async_global();       // the partials are read back by bulk copies
     if (!ok) {

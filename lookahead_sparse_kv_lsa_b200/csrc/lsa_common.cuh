@@ -190,6 +190,20 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
   return v;
 }
 
+// The one spin-wait of the grid barriers: until *counter >= target (acquire, gpu scope).
+// Gives up and returns false after limit_ns, or after an iteration count that the sleep
+// between polls makes longer than limit_ns (a second bound, should the timer stall).
+__device__ __forceinline__ bool spin_until_geq(const unsigned int* counter, unsigned int target,
+                                               uint64_t limit_ns = LSA_WAIT_LIMIT_NS) {
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t max_polls = limit_ns / 16u + 1024u;
+  for (uint64_t it = 0; ld_acquire_gpu(counter) < target; ++it) {
+    __nanosleep(32);
+    if (globaltimer_ns() - t0 > limit_ns || it > max_polls) return false;
+  }
+  return true;
+}
+
 // Plain shared stores (volatile: kept in order with the fences and barriers that
 // follow them; no memory clobber, so surrounding loads may still be scheduled freely).
 __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {

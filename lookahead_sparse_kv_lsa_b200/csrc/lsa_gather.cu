@@ -153,16 +153,9 @@ __device__ __forceinline__ void delta_sync(const DeltaArgs& a, int* abort, unsig
     __threadfence();
     atomicAdd(a.sync, 1u);
     const unsigned int target = k * gridDim.x;
-    if (!*abort) {
-      const uint64_t t0 = globaltimer_ns();
-      while (ld_acquire_gpu(a.sync) < target) {
-        __nanosleep(64);
-        if (globaltimer_ns() - t0 > LSA_WAIT_LIMIT_NS) {
-          set_err(a.g.err, LSA_DEVERR_TIMEOUT);
-          *abort = 1;
-          break;
-        }
-      }
+    if (!*abort && !spin_until_geq(a.sync, target)) {
+      set_err(a.g.err, LSA_DEVERR_TIMEOUT);
+      *abort = 1;
     }
     __threadfence();
   }

@@ -189,16 +189,9 @@ __device__ __forceinline__ void grid_sync(const Args& a, Smem* s, unsigned int k
     __threadfence();
     atomicAdd(a.sync, 1u);
     const unsigned int target = k * gridDim.x;
-    if (!s->abort) {
-      const uint64_t t0 = globaltimer_ns();
-      while (ld_acquire_gpu(a.sync) < target) {
-        __nanosleep(32);
-        if (globaltimer_ns() - t0 > LSA_WAIT_LIMIT_NS) {
-          set_err(a.err, LSA_DEVERR_TIMEOUT);
-          s->abort = 1;
-          break;
-        }
-      }
+    if (!s->abort && !spin_until_geq(a.sync, target)) {
+      set_err(a.err, LSA_DEVERR_TIMEOUT);
+      s->abort = 1;
     }
     __threadfence();
   }

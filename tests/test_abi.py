@@ -91,4 +91,8 @@ def test_invalid_arguments_rejected_before_device_work(lib):
                                       a["ids"], a["cap"], fake, fake, a["ws"], fake,
                                       None) == _lib.LSA_ERR_INVALID_ARG, bad
     assert lib.lsa_denoise_workspace_size(64) == 256
+    # the bounded-wait self-test: a flag and an error word, 1 ns .. 10 s
+    assert lib.lsa_wait_selftest(None, 1, 1000, fake, None) == _lib.LSA_ERR_INVALID_ARG
+    assert lib.lsa_wait_selftest(fake, 1, 0, fake, None) == _lib.LSA_ERR_INVALID_ARG
+    assert lib.lsa_wait_selftest(fake, 1, 10**10 + 1, fake, None) == _lib.LSA_ERR_INVALID_ARG
     assert lib.lsa_denoise_workspace_size(65) == 512
