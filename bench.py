@@ -560,11 +560,10 @@ def denoise_report(dev, hbm, with_oracle=True, reps=20):
     label_mask = torch.empty((W, NW), dtype=torch.int32, device=dev)
     label_ids = torch.empty((W, cap), dtype=torch.int32, device=dev)
     label_cnt = torch.empty((W,), dtype=torch.int32, device=dev)
-    ws = torch.zeros(lsa.denoise_workspace_size(W), dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def launch(i):
-        lsa.lsa_denoise_labels(copies[i % 3], set_mask, label_cnt, ws, err, top_p=cfg.top_p,
+        lsa.lsa_denoise_labels(copies[i % 3], set_mask, label_cnt, err, top_p=cfg.top_p,
                                min_votes=cfg.min_votes, set_cnt=set_cnt,
                                label_mask=label_mask, label_ids=label_ids)
     for i in range(3):

@@ -372,22 +372,19 @@ lsa_status lsa_wait_selftest(const uint32_t* flag, uint32_t target, int64_t limi
  *   label_ids   device i32 [n_windows][label_cap] out: the labels in increasing id, the
  *               first label_cap of them (may be null when label_cap == 0)
  *   label_cnt   device i32 [n_windows] out: the number of labels (may exceed label_cap)
- *   ws          device workspace of lsa_denoise_workspace_size(n_windows) bytes,
- *               4-byte aligned, zeroed before the first call (per-window counters that
- *               every call leaves at zero)
  * Supported: 1 <= n_layers <= 63, 1 <= n_blocks <= LSA_DENOISE_MAX_BLOCKS,
  * 0 < top_p <= 1; any min_votes (<= 0 keeps every block, > n_layers none).
  * Ties in probability are ties in the fp32 logit, so the tie order is exact; where the
  * running mass meets top_p within rounding (fp32 probabilities, fp64 sums) the boundary
- * block may differ from an exact computation. One launch, one CTA per (window, layer).
+ * block may differ from an exact computation. Two launches on `stream`: one CTA per
+ * (window, layer) for the sets, then one CTA per window for the vote.
  */
 #define LSA_DENOISE_MAX_BLOCKS 45056
 lsa_status lsa_denoise_labels(const float* logits, int32_t n_windows, int32_t n_layers,
                               int32_t n_blocks, double top_p, int32_t min_votes,
                               uint32_t* set_mask, int32_t* set_cnt, uint32_t* label_mask,
                               int32_t* label_ids, int32_t label_cap, int32_t* label_cnt,
-                              void* ws, size_t ws_bytes, int32_t* err, void* stream);
-size_t lsa_denoise_workspace_size(int32_t n_windows);
+                              int32_t* err, void* stream);
 
 #ifdef __cplusplus
 }

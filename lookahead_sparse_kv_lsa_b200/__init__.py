@@ -16,7 +16,7 @@ from ._lib import LsaError, LsaState, BLOCK, TAU
 
 __all__ = ["lsa_index", "lsa_gather", "lsa_gather_delta", "lsa_decode_attn", "lsa_step",
            "lsa_load_window", "gather_delta_workspace_size", "lsa_denoise_labels",
-           "denoise_workspace_size", "DENOISE_MAX_BLOCKS", "lsa_wait_selftest",
+           "DENOISE_MAX_BLOCKS", "lsa_wait_selftest",
            "lsa_pass_setup", "lsa_append", "lsa_decode_step",
            "index_workspace_size", "decode_attn_workspace_size", "LsaDecoder", "LsaError",
            "LsaState", "BLOCK", "TAU", "library_path"]
@@ -138,16 +138,12 @@ def lsa_gather_delta(host_pool, host_blk_off, sel_ids, sel_cnt, res_pages, n_res
 DENOISE_MAX_BLOCKS = 45056
 
 
-def denoise_workspace_size(n_windows: int) -> int:
-    return int(_lib.lib().lsa_denoise_workspace_size(n_windows))
-
-
-def lsa_denoise_labels(logits, set_mask, label_cnt, ws, err, top_p: float = 0.6,
+def lsa_denoise_labels(logits, set_mask, label_cnt, err, top_p: float = 0.6,
                        min_votes: int = 3, set_cnt=None, label_mask=None, label_ids=None,
                        stream=None) -> None:
     """Label denoising (lsa_denoise_labels in lsa.h). logits: f32 [W][L][N] on the device;
     set_mask: u32 words [W][L][ceil(N/32)] (an int32 tensor); label_cnt: i32 [W];
-    label_ids: i32 [W][cap] or None; ws: zero-filled uint8 of denoise_workspace_size(W)."""
+    label_ids: i32 [W][cap] or None."""
     W, L, N = logits.shape
     NW = (N + 31) // 32
     cap = 0 if label_ids is None else label_ids.shape[1]
@@ -157,8 +153,8 @@ def lsa_denoise_labels(logits, set_mask, label_cnt, ws, err, top_p: float = 0.6,
         _opt(set_cnt, torch.int32, "set_cnt", W * L),
         _opt(label_mask, torch.int32, "label_mask", W * NW),
         _opt(label_ids, torch.int32, "label_ids", W * cap), cap,
-        _dev(label_cnt, torch.int32, "label_cnt", W), _dev(ws, torch.uint8, "ws"), ws.numel(),
-        _dev(err, torch.int32, "err", 1), _stream(stream))
+        _dev(label_cnt, torch.int32, "label_cnt", W), _dev(err, torch.int32, "err", 1),
+        _stream(stream))
     _lib.check("lsa_denoise_labels", st)
 
 

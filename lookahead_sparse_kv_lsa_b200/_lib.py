@@ -77,8 +77,7 @@ SIGNATURES = {
     "lsa_append": (_i32, [C.POINTER(LsaState), _i64, _p, _p, _p]),
     "lsa_decode_step": (_i32, [C.POINTER(LsaState), _i64, _p, _p, _p, _p, _p]),
     "lsa_denoise_labels": (_i32, [_p, _i32, _i32, _i32, C.c_double, _i32, _p, _p, _p, _p, _i32,
-                                  _p, _p, _sz, _p, _p]),
-    "lsa_denoise_workspace_size": (_sz, [_i32]),
+                                  _p, _p, _p]),
     "lsa_wait_selftest": (_i32, [_p, C.c_uint32, _i64, _p, _p]),
 }
 

@@ -27,8 +27,8 @@
 //
 // In the first pass each thread accumulates its share of the histogram in its own
 // shared-memory column (bank = lane), so the mass needs no shared atomics; the bins are
-// summed in fp64. The vote runs in the last CTA of each window (a per-window ticket in
-// the workspace), as bit-sliced counters over the layers' 32-block mask words.
+// summed in fp64. The vote is a second launch, one CTA per window, as bit-sliced counters
+// over the layers' 32-block mask words.
 #include "lsa_common.cuh"
 
 namespace lsa {
@@ -54,7 +54,6 @@ struct DenoiseArgs {
   int32_t* label_ids;    // [W][label_cap]
   int32_t label_cap;
   int32_t* label_cnt;    // [W]
-  uint32_t* tickets;     // [W], zero between calls
   int32_t* err;
 };
 
@@ -539,9 +538,8 @@ __device__ __noinline__ void resolve_list(const DenoiseArgs& a, float ml2, doubl
 }
 
 // ---------------------------------------------------------------- the window's vote
-// Run by the window's last CTA: bit-sliced counters over the L mask words of each
-// 32-block group, labels written as a mask and as increasing ids. `lab` is shared
-// scratch of NW words.
+// Bit-sliced counters over the L mask words of each 32-block group of window w, labels
+// written as a mask and as increasing ids. `lab` is shared scratch of NW words.
 __device__ __noinline__ void vote_window(const DenoiseArgs& a, int w, uint32_t* lab) {
   Smem& s = sm();
   const int tid = threadIdx.x;
@@ -606,10 +604,7 @@ __device__ __noinline__ void vote_window(const DenoiseArgs& a, int w, uint32_t* 
       b &= b - 1u;
     }
   }
-  if (tid == 0) {
-    a.label_cnt[w] = total;
-    a.tickets[w] = 0u;  // ready for the next call
-  }
+  if (tid == 0) a.label_cnt[w] = total;
   (void)s;
 }
 
@@ -622,7 +617,6 @@ __global__ void __launch_bounds__(NT, 2) denoise_kernel(const __grid_constant__ 
   uint32_t* bw = bin_words(NW);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x;
-  const int w = row / a.L;
   const float* src = a.logits + static_cast<size_t>(row) * N;
 
   // ---- the row into shared memory; the row max
@@ -730,22 +724,25 @@ __global__ void __launch_bounds__(NT, 2) denoise_kernel(const __grid_constant__ 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
 
-  // ---- the row's set size, the window ticket, the vote when this row closes the window
+  // ---- the row's set size
   if (lane == 0) s.wcnt[warp] = cnt;
   __syncthreads();
-  if (tid == 0) {
+  if (tid == 0 && a.set_cnt) {
     int t = 0;
     for (int k = 0; k < NWARP; ++k) t += s.wcnt[k];
-    if (a.set_cnt) a.set_cnt[row] = t;
-    // the CTA's mask stores, ordered before this thread by the barrier, become visible
-    // device-wide before the ticket (fence cumulativity)
-    __threadfence();
-    s.last = atomicAdd(&a.tickets[w], 1u) == static_cast<uint32_t>(a.L - 1);
+    a.set_cnt[row] = t;
   }
-  __syncthreads();
-  if (!s.last) return;
-  __threadfence();
-  vote_window(a, w, bw);  // the bin words are scratch now
+}
+
+// The vote, one CTA per window, launched after denoise_kernel on the same stream (so all
+// the window's set masks are complete): shared memory is Smem, then NW words of scratch.
+__global__ void __launch_bounds__(NT, 1) vote_kernel(const __grid_constant__ DenoiseArgs a) {
+  // no row here: the scratch words follow Smem directly (vote_smem_bytes)
+  vote_window(a, blockIdx.x, reinterpret_cast<uint32_t*>(dn_smem + sizeof(Smem)));
+}
+
+size_t vote_smem_bytes(int32_t NW) {
+  return sizeof(Smem) + static_cast<size_t>(NW) * sizeof(uint32_t);
 }
 
 size_t smem_bytes(int32_t NW) {
@@ -763,35 +760,28 @@ static_assert(DN_CAND <= NT, "one scan lane per ranked candidate");
 }  // namespace
 }  // namespace lsa
 
-extern "C" size_t lsa_denoise_workspace_size(int32_t n_windows) {
-  if (n_windows <= 0) return 0;
-  return (static_cast<size_t>(n_windows) * sizeof(uint32_t) + 255u) / 256u * 256u;
-}
-
 extern "C" lsa_status lsa_denoise_labels(const float* logits, int32_t n_windows,
                                          int32_t n_layers, int32_t n_blocks, double top_p,
                                          int32_t min_votes, uint32_t* set_mask,
                                          int32_t* set_cnt, uint32_t* label_mask,
                                          int32_t* label_ids, int32_t label_cap,
-                                         int32_t* label_cnt, void* ws, size_t ws_bytes,
-                                         int32_t* err, void* stream) {
+                                         int32_t* label_cnt, int32_t* err, void* stream) {
   using namespace lsa;
-  if (logits == nullptr || set_mask == nullptr || label_cnt == nullptr || ws == nullptr)
-    return LSA_ERR_INVALID_ARG;
+  if (logits == nullptr || set_mask == nullptr || label_cnt == nullptr) return LSA_ERR_INVALID_ARG;
   if (n_windows < 1 || n_layers < 1 || n_layers >= (1 << DN_PLANES) || n_blocks < 1 ||
       n_blocks > LSA_DENOISE_MAX_BLOCKS)
     return LSA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(n_windows) * n_layers > 0x7fffffffLL) return LSA_ERR_INVALID_ARG;
   if (!(top_p > 0.0) || !(top_p <= 1.0)) return LSA_ERR_INVALID_ARG;
   if (label_cap < 0 || (label_cap > 0 && label_ids == nullptr)) return LSA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(ws) & 3u) != 0 ||
-      ws_bytes < lsa_denoise_workspace_size(n_windows))
-    return LSA_ERR_INVALID_ARG;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(denoise_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem_bytes(LSA_DENOISE_MAX_BLOCKS / 32))) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(vote_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(vote_smem_bytes(LSA_DENOISE_MAX_BLOCKS / 32))) !=
+            cudaSuccess)
       return LSA_ERR_CUDA;
     attr = true;
   }
@@ -809,8 +799,10 @@ extern "C" lsa_status lsa_denoise_labels(const float* logits, int32_t n_windows,
   a.label_ids = label_ids;
   a.label_cap = label_cap;
   a.label_cnt = label_cnt;
-  a.tickets = static_cast<uint32_t*>(ws);
   a.err = err;
-  denoise_kernel<<<n_windows * n_layers, NT, smem_bytes(a.NW), static_cast<cudaStream_t>(stream)>>>(a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  denoise_kernel<<<n_windows * n_layers, NT, smem_bytes(a.NW), st>>>(a);
+  if (cudaPeekAtLastError() != cudaSuccess) return LSA_ERR_CUDA;
+  vote_kernel<<<n_windows, NT, vote_smem_bytes(a.NW), st>>>(a);
   return cudaPeekAtLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
 }

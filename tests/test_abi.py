@@ -81,18 +81,15 @@ def test_invalid_arguments_rejected_before_device_work(lib):
     st = _lib.LsaState()
     assert lib.lsa_state_check(C.byref(st)) == _lib.LSA_ERR_INVALID_ARG
     assert lib.lsa_step(None, 0, None, None, None, None, None, None) == _lib.LSA_ERR_INVALID_ARG
-    # label denoising: layers 1..63, blocks 1..45056, 0 < top_p <= 1, ids when cap > 0,
-    # a workspace of one counter per window
-    ok = dict(W=4, L=21, N=1000, p=0.6, cap=8, ids=fake, ws=1024)
+    # label denoising: layers 1..63, blocks 1..45056, 0 < top_p <= 1, ids when cap > 0
+    ok = dict(W=4, L=21, N=1000, p=0.6, cap=8, ids=fake, logits=fake)
     for bad in (dict(L=0), dict(L=64), dict(N=0), dict(N=45057), dict(p=0.0), dict(p=1.5),
-                dict(p=float("nan")), dict(cap=-1), dict(ids=None), dict(ws=8), dict(W=0)):
+                dict(p=float("nan")), dict(cap=-1), dict(ids=None), dict(W=0), dict(logits=None)):
         a = dict(ok, **bad)
-        assert lib.lsa_denoise_labels(fake, a["W"], a["L"], a["N"], a["p"], 3, fake, None, None,
-                                      a["ids"], a["cap"], fake, fake, a["ws"], fake,
+        assert lib.lsa_denoise_labels(a["logits"], a["W"], a["L"], a["N"], a["p"], 3, fake, None,
+                                      None, a["ids"], a["cap"], fake, fake,
                                       None) == _lib.LSA_ERR_INVALID_ARG, bad
-    assert lib.lsa_denoise_workspace_size(64) == 256
     # the bounded-wait self-test: a flag and an error word, 1 ns .. 10 s
     assert lib.lsa_wait_selftest(None, 1, 1000, fake, None) == _lib.LSA_ERR_INVALID_ARG
     assert lib.lsa_wait_selftest(fake, 1, 0, fake, None) == _lib.LSA_ERR_INVALID_ARG
     assert lib.lsa_wait_selftest(fake, 1, 10**10 + 1, fake, None) == _lib.LSA_ERR_INVALID_ARG
-    assert lib.lsa_denoise_workspace_size(65) == 512
