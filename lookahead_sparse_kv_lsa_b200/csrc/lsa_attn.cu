@@ -884,9 +884,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float p = (valid && h < a.H) ? exp2f(fmaf(s[h], a.scale_log2, -mu)) : 0.f;
             // the denominator sums the same bf16-rounded weights that multiply V, so the
             // output stays a normalised average of V rows (exact for a one-hot softmax)
-            const float pr = __bfloat162float(__float2bfloat16_rn(p));
-            lp[h] = lp[h] * al + pr;
-            s[h] = pr;
+            const __nv_bfloat16 pb = __float2bfloat16_rn(p);
+            lp[h] = lp[h] * al + __bfloat162float(pb);
+            s[h] = __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(pb)));  // bits kept
           }
           // the previous tile's P . V must be done before P is overwritten or O rescaled
           if (gtile_o >= 1)
@@ -914,10 +914,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             uint8_t* pc = sP + (row >> 6) * HP * 128;
             const uint32_t byte_in_row = (row & 63) * 2;
 #pragma unroll
-            for (int h = 0; h < HP; ++h) {
-              const __nv_bfloat16 v = __float2bfloat16_rn(s[h]);
-              *reinterpret_cast<__nv_bfloat16*>(pc + sw128_offset(h, byte_in_row)) = v;
-            }
+            for (int h = 0; h < HP; ++h)
+              *reinterpret_cast<uint16_t*>(pc + sw128_offset(h, byte_in_row)) =
+                  static_cast<uint16_t>(__float_as_uint(s[h]));
           }
           fence_proxy_async_smem();
           tc_fence_before();
