@@ -216,6 +216,15 @@ __device__ __forceinline__ void store_scattered(float* dst, const float (&v)[N],
   }
 }
 
+// 2^x on the special-function unit (relative error about 2^-22, results below 2^-126
+// flushed to zero): the softmax weights are rounded to bf16 right after, so the extra
+// care of exp2f for subnormal results buys nothing.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // TMEM load of HP consecutive columns of this warp's 32 lanes.
 template <int HP>
 __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[HP]) {
@@ -881,7 +890,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float mu = m->m_use[h];
             const float al = m->alpha[h];
             rescale |= al < 1.f;
-            const float p = (valid && h < a.H) ? exp2f(fmaf(s[h], a.scale_log2, -mu)) : 0.f;
+            const float p = (valid && h < a.H) ? ex2_approx(fmaf(s[h], a.scale_log2, -mu)) : 0.f;
             // the denominator sums the same bf16-rounded weights that multiply V, so the
             // output stays a normalised average of V rows (exact for a one-hot softmax)
             const __nv_bfloat16 pb = __float2bfloat16_rn(p);
