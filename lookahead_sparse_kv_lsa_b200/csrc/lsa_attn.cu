@@ -60,6 +60,7 @@ struct Misc {
   float red[4][64];
   float m_use[64];
   float alpha[64];
+  int resc_tile;                    // the last softmax tile in which some head rescaled
   // fused merge
   int n_items, total_items;
   long long merge_j0, merge_j1, cur_j;
@@ -631,6 +632,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&m->q_free, 1);
     mbar_init(&m->mma_done, 1);
     m->abort = 0;
+    m->resc_tile = -1;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -872,6 +874,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (h < a.H && mt > m_run + RESCALE_LOG2) {
               al = exp2f(m_run - mt);          // 0 when nothing was accumulated yet
               m_run = mt;
+              m->resc_tile = gtile_s;          // the same value from every head that rescales
             }
             m->m_use[h] = m_run;
             m->alpha[h] = al;
@@ -884,18 +887,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&m->s_free[sb]);
           ++gtile_s;
-          bool rescale = false;
+          // gtile_s was advanced above: the tile whose alphas were just set is gtile_s - 1
+          const bool rescale = m->resc_tile == gtile_s - 1;
+          // The denominator sums the same bf16-rounded weights that multiply V, so the
+          // output stays a normalised average of V rows (exact for a one-hot softmax); the
+          // rounded bits are kept for the P operand.
+          if (!rescale && a.H == HP && __all_sync(0xffffffffu, valid)) {
+            // common case: no head rescales, every row and head is live
 #pragma unroll
-          for (int h = 0; h < HP; ++h) {
-            const float mu = m->m_use[h];
-            const float al = m->alpha[h];
-            rescale |= al < 1.f;
-            const float p = (valid && h < a.H) ? ex2_approx(fmaf(s[h], a.scale_log2, -mu)) : 0.f;
-            // the denominator sums the same bf16-rounded weights that multiply V, so the
-            // output stays a normalised average of V rows (exact for a one-hot softmax)
-            const __nv_bfloat16 pb = __float2bfloat16_rn(p);
-            lp[h] = lp[h] * al + __bfloat162float(pb);
-            s[h] = __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(pb)));  // bits kept
+            for (int h = 0; h < HP; ++h) {
+              const float p = ex2_approx(fmaf(s[h], a.scale_log2, -m->m_use[h]));
+              const __nv_bfloat16 pb = __float2bfloat16_rn(p);
+              lp[h] += __bfloat162float(pb);
+              s[h] = __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(pb)));
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < HP; ++h) {
+              const float mu = m->m_use[h];
+              const float al = m->alpha[h];
+              const float p = (valid && h < a.H) ? ex2_approx(fmaf(s[h], a.scale_log2, -mu)) : 0.f;
+              const __nv_bfloat16 pb = __float2bfloat16_rn(p);
+              lp[h] = lp[h] * al + __bfloat162float(pb);
+              s[h] = __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(pb)));
+            }
           }
           // the previous tile's P . V must be done before P is overwritten or O rescaled
           if (gtile_o >= 1)
