@@ -857,8 +857,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float x[HP];
             tmem_ld_row<HP>(tmem + lane_addr + sb * HP, x);
             tmem_wait_ld();
+            if (!__all_sync(0xffffffffu, valid)) {
 #pragma unroll
-            for (int h = 0; h < HP; ++h) x[h] = valid ? x[h] : -INFINITY;
+              for (int h = 0; h < HP; ++h) x[h] = valid ? x[h] : -INFINITY;
+            }
             warp_reduce_scatter<HP, true>(x, lane);
             store_scattered<HP>(m->red[sw], x, lane);
           }
@@ -895,11 +897,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!rescale && a.H == HP && __all_sync(0xffffffffu, valid)) {
             // common case: no head rescales, every row and head is live
 #pragma unroll
-            for (int h = 0; h < HP; ++h) {
-              const float p = ex2_approx(fmaf(s[h], a.scale_log2, -m->m_use[h]));
-              const __nv_bfloat16 pb = __float2bfloat16_rn(p);
-              lp[h] += __bfloat162float(pb);
-              s[h] = __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(pb)));
+            for (int h = 0; h < HP; h += 2) {
+              const float p0 = ex2_approx(fmaf(s[h], a.scale_log2, -m->m_use[h]));
+              const float p1 = ex2_approx(fmaf(s[h + 1], a.scale_log2, -m->m_use[h + 1]));
+              // both weights rounded by one conversion: p0 in the low half, p1 in the high
+              const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+              const uint32_t w = *reinterpret_cast<const uint32_t*>(&pb);
+              lp[h] += __uint_as_float(w << 16);
+              lp[h + 1] += __uint_as_float(w & 0xffff0000u);
+              s[h] = __uint_as_float(w & 0xffffu);
+              s[h + 1] = __uint_as_float(w >> 16);
             }
           } else {
 #pragma unroll
