@@ -85,8 +85,10 @@ int32_t lsa_version(void);
  *   layer_mask nullable device u32 [L+1][B][ceil(max_cand/32)] out: bit c%32 of word
  *             c/32 = (z_l > 0) for l < L, and the OR for l = L
  *   ws        device workspace of lsa_index_workspace_size(B, L, d_i, max_cand) bytes,
- *             16-byte aligned, zero-filled before the first call (every call leaves its
- *             grid-barrier counters zero again)
+ *             16-byte aligned, zero-filled before the first call. Its first 8 bytes are
+ *             a grid-barrier counter that grows by twice the grid size per call; the
+ *             caller must not change them between calls. A workspace sized for one shape
+ *             serves any shape whose size is no larger, on the same device.
  * Supported: 1 <= L <= 4, d_i == 128, D % 256 == 0, B >= 1, cap >= 0. One cooperative
  * launch (one CTA per SM, all resident) with two grid-wide barriers: projection, then
  * scoring, then compaction.

@@ -8,8 +8,9 @@
 //
 // One cooperative launch, one CTA per SM, three phases split by two grid barriers:
 //
-//  A. Warp 0 starts 16-byte asynchronous copies of the CTA's share of K_idx into
-//     shared memory (it does not depend on q); warps 1.. compute the CTA's share of the
+//  A. Warp 0 plans the CTA's share of K_idx rows and four copy warps start their 16-byte
+//     asynchronous copies into shared memory (they do not depend on q); the other warps
+//     compute the CTA's share of the
 //     W_q rows: q[l][b][j] = W_q[l][j] . h[l][b] in fp32, each dot cut into four fixed
 //     parts summed in a fixed order.
 //  B. Scoring. The candidate rows of every sequence are grouped in 32-row "words"; all
@@ -22,8 +23,8 @@
 //     words of the same sequence, a block scan over its own) and writes the ascending id
 //     list; the CTA holding a sequence's last word writes its count.
 //
-// Grid barriers use an arrival counter in the workspace with a bounded wait; the last
-// CTA to leave resets the counters, so the workspace is left as it was found (zero).
+// Grid barriers use a 64-bit arrival counter in the workspace with a bounded wait. The
+// counter only grows (by 2 x grid per launch), so no CTA has to reset it on the way out.
 #include "lsa_common.cuh"
 
 namespace lsa {
@@ -44,6 +45,7 @@ constexpr int NPART = 4;                            // projection: parts per dot
 constexpr int RMAX = 4;                             // projection: W_q rows per round
 constexpr int BCH = 32;                             // projection: sequences per round
 constexpr int MAX_GRID = 1024;
+constexpr int KW = 4;                               // warps that copy K_idx rows (named barrier 2)
 
 struct Args {
   const uint16_t* h;         // [L][B][D]
@@ -56,7 +58,7 @@ struct Args {
   const int32_t* n_cand;     // [B]
   float* q;                  // workspace [L][B][D_I]
   uint32_t* words;           // workspace [B][n_words]: OR keep bits
-  unsigned int* sync;        // workspace [2]: barrier arrivals, departures
+  unsigned long long* sync;  // workspace: grid-barrier arrivals (grows by 2 x grid per launch)
   int32_t* sel_ids;          // [B][cap]
   int32_t* sel_cnt;          // [B]
   float* logits;             // nullable [L][B][max_cand]
@@ -83,6 +85,7 @@ struct SeqTab {
 struct Smem {
   uint8_t kbuf[CHUNK_WORDS * WORD_SMEM];
   int abort;
+  uint32_t own[CHUNK_WORDS];             // keep words of the first chunk, as scored
   int word_seq[CHUNK_WORDS];             // table entry of each word of the chunk
   alignas(16) float qs[CHUNK_WORDS][MAX_L][D_I];   // queries of the chunk's sequences
   int red[NWARPS];
@@ -114,37 +117,47 @@ __device__ __forceinline__ int seq_cand(const Args& a, int b, bool report) {
 }
 __device__ __forceinline__ int seq_words(int n) { return (n + WORD_ROWS - 1) / WORD_ROWS; }
 
-__device__ __forceinline__ void prefetch_l1(const void* p) {
-  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
-}
+// Candidate count, K_idx offset and bias of sequence `lane` (< 32), loaded together.
+struct SeqHead {
+  int n;
+  long long row0;
+  float bias;
+};
 
 // Total keep words of the batch, summed by one warp (every lane gets it). The first 32
-// sequences' K_idx offsets and biases, which the plan reads next, are prefetched.
-__device__ __forceinline__ long long warp_total_words(const Args& a, int lane) {
+// sequences' counts, K_idx offsets and biases, which the plan reads next, are loaded in
+// the same round trip and returned in `head`.
+__device__ __forceinline__ long long warp_total_words(const Args& a, int lane, SeqHead& head) {
+  head.n = 0;
+  head.row0 = 0;
+  head.bias = 0.f;
   if (lane < a.B) {
-    prefetch_l1(a.kidx_off + lane);
-    prefetch_l1(a.bias + lane);
+    head.n = seq_cand(a, lane, false);
+    head.row0 = __ldg(a.kidx_off + lane);
+    head.bias = __ldg(a.bias + lane);
   }
-  long long s = 0;
-  for (int b = lane; b < a.B; b += 32) s += seq_words(seq_cand(a, b, false));
+  long long s = seq_words(head.n);
+  for (int b = lane + 32; b < a.B; b += 32) s += seq_words(seq_cand(a, b, false));
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   return s;
 }
 
 // Warp 0: fill t with the sequences that own words of [w_lo, w_hi), walking forward
-// from the saved state (sequence resume_b, whose first word is resume_base).
+// from the saved state (sequence resume_b, whose first word is resume_base). `head`, if
+// given, holds sequence `lane`'s count, offset and bias (the walk's first 32 sequences).
 __device__ __forceinline__ void plan_words(const Args& a, long long w_lo, long long w_hi, SeqTab* t,
-                                          int lane) {
+                                          int lane, const SeqHead* head = nullptr) {
   int found = 0;
   long long base = t->resume_base;
   int last_b = t->resume_b;
   long long last_base = t->resume_base;
   for (int b0 = t->resume_b; b0 < a.B && base < w_hi; b0 += 32) {
     const int b = b0 + lane;
-    const int n = b < a.B ? seq_cand(a, b, false) : 0;
-    const long long row0 = b < a.B ? __ldg(a.kidx_off + b) : 0;   // loaded with n
-    const float bias = b < a.B ? __ldg(a.bias + b) : 0.f;
+    const bool pre = head != nullptr && b0 == 0;
+    const int n = pre ? head->n : (b < a.B ? seq_cand(a, b, false) : 0);
+    const long long row0 = pre ? head->row0 : (b < a.B ? __ldg(a.kidx_off + b) : 0);
+    const float bias = pre ? head->bias : (b < a.B ? __ldg(a.bias + b) : 0.f);
     const int nw = seq_words(n);
     long long incl = nw;
 #pragma unroll
@@ -181,15 +194,35 @@ __device__ __forceinline__ void plan_words(const Args& a, long long w_lo, long l
   }
 }
 
-// Grid-wide barrier number k (1, 2, ...): every CTA arrives; the wait is bounded and,
-// once the CTA has given up (abort), it still arrives but no longer waits.
-__device__ __forceinline__ void grid_sync(const Args& a, Smem* s, unsigned int k) {
+// Bounded spin until the 64-bit *counter >= target (acquire, gpu scope), with the same
+// two limits as the 32-bit spin_until_geq: the timer and an iteration count that the
+// sleep between polls makes longer than limit_ns.
+__device__ __forceinline__ bool spin_until_geq64(const unsigned long long* counter,
+                                                 unsigned long long target,
+                                                 uint64_t limit_ns = LSA_WAIT_LIMIT_NS) {
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t max_polls = limit_ns / 16u + 1024u;
+  for (uint64_t it = 0;; ++it) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(counter) : "memory");
+    if (v >= target) return true;
+    __nanosleep(32);
+    if (globaltimer_ns() - t0 > limit_ns || it > max_polls) return false;
+  }
+}
+
+// Grid-wide barrier on a 64-bit arrival counter that only grows: every launch adds
+// exactly 2 x gridDim.x (each CTA arrives at both barriers, also after giving up), so at
+// a barrier the count it must reach is the next multiple of gridDim.x above the value
+// this CTA's arrival saw. Nothing has to reset the counter after the launch. The wait is
+// bounded; once the CTA has given up (abort) it still arrives but no longer waits.
+__device__ __forceinline__ void grid_sync(const Args& a, Smem* s) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
-    atomicAdd(a.sync, 1u);
-    const unsigned int target = k * gridDim.x;
-    if (!s->abort && !spin_until_geq(a.sync, target)) {
+    const unsigned long long seen = atomicAdd(a.sync, 1ull);
+    const unsigned long long target = (seen / gridDim.x + 1ull) * gridDim.x;
+    if (!s->abort && !spin_until_geq64(a.sync, target)) {
       set_err(a.err, LSA_DEVERR_TIMEOUT);
       s->abort = 1;
     }
@@ -198,12 +231,10 @@ __device__ __forceinline__ void grid_sync(const Args& a, Smem* s, unsigned int k
   __syncthreads();
 }
 
-// Warp 0: plan the chunk [cw0, cw1) of keep words and start the 16-byte asynchronous
-// copies of their K_idx rows into s->kbuf (padded rows; a sequence's last word may be
-// partial). Completed by cp_async_wait_all in the same warp.
-__device__ __forceinline__ void issue_chunk(const Args& a, Smem* s, long long cw0, long long cw1,
-                                            int lane) {
-  plan_words(a, cw0, cw1, &s->tab, lane);
+// Warp 0: plan the chunk [cw0, cw1) of keep words into s->tab and s->word_seq.
+__device__ __forceinline__ void plan_chunk(const Args& a, Smem* s, long long cw0, long long cw1,
+                                           int lane, const SeqHead* head = nullptr) {
+  plan_words(a, cw0, cw1, &s->tab, lane, head);
   __syncwarp();
   const int nwc = static_cast<int>(cw1 - cw0);
   if (lane < nwc) {
@@ -212,7 +243,14 @@ __device__ __forceinline__ void issue_chunk(const Args& a, Smem* s, long long cw
     while (i + 1 < s->tab.n && s->tab.w0[i + 1] <= w) ++i;
     s->word_seq[lane] = i;
   }
-  __syncwarp();
+}
+
+// Copy warps (thread ct of KW * 32): start the 16-byte asynchronous copies of the planned
+// chunk's K_idx rows into s->kbuf (padded rows; a sequence's last word may be partial).
+// Each copy warp completes its own copies with cp_async_wait_all.
+__device__ __forceinline__ void copy_chunk(const Args& a, Smem* s, long long cw0, long long cw1,
+                                           int ct) {
+  const int nwc = static_cast<int>(cw1 - cw0);
   for (int k = 0; k < nwc; ++k) {
     const int i = s->word_seq[k];
     const int wi = static_cast<int>(cw0 + k - s->tab.w0[i]);
@@ -221,7 +259,7 @@ __device__ __forceinline__ void issue_chunk(const Args& a, Smem* s, long long cw
       const uint8_t* src = reinterpret_cast<const uint8_t*>(
           a.k_idx + (t * a.kls + s->tab.row0[i] + static_cast<long long>(WORD_ROWS) * wi) * D_I);
       const uint32_t dst = smem_u32(s->kbuf + (k * a.lk + t) * WORD_SMEM);
-      for (int p = lane; p < rows * (ROW_BYTES / 16); p += 32) {
+      for (int p = ct; p < rows * (ROW_BYTES / 16); p += KW * 32) {
         const int r = p >> 4, c = p & 15;
         cp_async16(dst + r * ROW_STRIDE + c * 16, src + r * ROW_BYTES + c * 16);
       }
@@ -247,9 +285,11 @@ __device__ __forceinline__ void stage_queries(const Args& a, Smem* s) {
 // Warp: keep word k of the current chunk, one lane per candidate row. The row's 16
 // pieces of 8 elements are read from its padded shared-memory row, the queries' pieces
 // are shared-memory broadcasts; each layer's dot product runs in two interleaved chains
-// joined in a fixed order. One ballot per layer gives the word's keep bits.
-template <bool PER_LAYER>
-__device__ __forceinline__ void score_word(const Args& a, Smem* s, int k, long long cw0, int lane) {
+// joined in a fixed order. One ballot per layer gives the word's keep bits; the OR over
+// the NL (= L) layers is returned. NL is a template argument so that the layers' chains
+// form one straight-line block the scheduler can interleave.
+template <bool PER_LAYER, int NL>
+__device__ __forceinline__ uint32_t score_word(const Args& a, Smem* s, int k, long long cw0, int lane) {
   const int i = s->word_seq[k];
   const int wi = static_cast<int>(cw0 + k - s->tab.w0[i]);
   const int c = WORD_ROWS * wi + lane;
@@ -257,63 +297,70 @@ __device__ __forceinline__ void score_word(const Args& a, Smem* s, int k, long l
   const float bias = s->tab.bias[i];
   const int b = s->tab.b[i];
   const uint8_t* rp = s->kbuf + k * a.lk * WORD_SMEM + lane * ROW_STRIDE;
-  float acc[MAX_L][2];
+  float acc[NL][2];
 #pragma unroll
-  for (int l = 0; l < MAX_L; ++l) acc[l][0] = acc[l][1] = 0.f;
+  for (int l = 0; l < NL; ++l) acc[l][0] = acc[l][1] = 0.f;
 #pragma unroll 4
   for (int j = 0; j < D_I / 8; ++j) {
     float kf[8];
     if (!PER_LAYER) unpack8(*reinterpret_cast<const uint4*>(rp + 16 * j), kf);
 #pragma unroll
-    for (int l = 0; l < MAX_L; ++l) {
-      if (l < a.L) {
-        if (PER_LAYER) unpack8(*reinterpret_cast<const uint4*>(rp + l * WORD_SMEM + 16 * j), kf);
-        const float4 qa = *reinterpret_cast<const float4*>(&s->qs[i][l][8 * j]);
-        const float4 qb = *reinterpret_cast<const float4*>(&s->qs[i][l][8 * j + 4]);
-        float& u = acc[l][j & 1];
-        u = fmaf(qa.x, kf[0], u);
-        u = fmaf(qa.y, kf[1], u);
-        u = fmaf(qa.z, kf[2], u);
-        u = fmaf(qa.w, kf[3], u);
-        u = fmaf(qb.x, kf[4], u);
-        u = fmaf(qb.y, kf[5], u);
-        u = fmaf(qb.z, kf[6], u);
-        u = fmaf(qb.w, kf[7], u);
-      }
+    for (int l = 0; l < NL; ++l) {
+      if (PER_LAYER) unpack8(*reinterpret_cast<const uint4*>(rp + l * WORD_SMEM + 16 * j), kf);
+      const float4 qa = *reinterpret_cast<const float4*>(&s->qs[i][l][8 * j]);
+      const float4 qb = *reinterpret_cast<const float4*>(&s->qs[i][l][8 * j + 4]);
+      float& u = acc[l][j & 1];
+      u = fmaf(qa.x, kf[0], u);
+      u = fmaf(qa.y, kf[1], u);
+      u = fmaf(qa.z, kf[2], u);
+      u = fmaf(qa.w, kf[3], u);
+      u = fmaf(qb.x, kf[4], u);
+      u = fmaf(qb.y, kf[5], u);
+      u = fmaf(qb.z, kf[6], u);
+      u = fmaf(qb.w, kf[7], u);
     }
   }
   uint32_t wor = 0;
-  uint32_t wl[MAX_L];
+  uint32_t wl[NL];
 #pragma unroll
-  for (int l = 0; l < MAX_L; ++l) {
-    wl[l] = 0u;
-    if (l < a.L) {
-      const float z = fmaf(acc[l][0] + acc[l][1], a.inv_sqrt_di, bias);
-      if (a.logits != nullptr && valid)
-        a.logits[(static_cast<long long>(l) * a.B + b) * a.max_cand + c] = z;
-      wl[l] = __ballot_sync(0xffffffffu, valid && z > 0.f);
-      wor |= wl[l];
-    }
+  for (int l = 0; l < NL; ++l) {
+    const float z = fmaf(acc[l][0] + acc[l][1], a.inv_sqrt_di, bias);
+    if (a.logits != nullptr && valid)
+      a.logits[(static_cast<long long>(l) * a.B + b) * a.max_cand + c] = z;
+    wl[l] = __ballot_sync(0xffffffffu, valid && z > 0.f);
+    wor |= wl[l];
   }
   if (lane == 0) {
     a.words[static_cast<long long>(b) * a.n_words + wi] = wor;
     if (a.layer_mask != nullptr) {
 #pragma unroll
-      for (int l = 0; l < MAX_L; ++l)
-        if (l < a.L) a.layer_mask[(static_cast<long long>(l) * a.B + b) * a.mask_words + wi] = wl[l];
-      a.layer_mask[(static_cast<long long>(a.L) * a.B + b) * a.mask_words + wi] = wor;
+      for (int l = 0; l < NL; ++l)
+        a.layer_mask[(static_cast<long long>(l) * a.B + b) * a.mask_words + wi] = wl[l];
+      a.layer_mask[(static_cast<long long>(NL) * a.B + b) * a.mask_words + wi] = wor;
     }
+  }
+  return wor;
+}
+
+template <bool PER_LAYER>
+__device__ __forceinline__ uint32_t score_word_any(const Args& a, Smem* s, int k, long long cw0,
+                                                   int lane) {
+  switch (a.L) {
+    case 1: return score_word<PER_LAYER, 1>(a, s, k, cw0, lane);
+    case 2: return score_word<PER_LAYER, 2>(a, s, k, cw0, lane);
+    case 3: return score_word<PER_LAYER, 3>(a, s, k, cw0, lane);
+    default: return score_word<PER_LAYER, MAX_L>(a, s, k, cw0, lane);
   }
 }
 
-// Warps 1.. (PROJ_THREADS threads, named barrier 1): q rows [r_lo, r_hi) of the stacked
+// Warps KW.. (PROJ_THREADS threads, named barrier 1): q rows [r_lo, r_hi) of the stacked
 // W_q (row = l * D_I + j) for every sequence. Each dot product is cut into NPART parts of
 // whole 8-element groups; a warp sums one part (lane-strided, then a butterfly), and the
 // parts are added in order.
-constexpr int PROJ_THREADS = NTHREADS - 32;
+constexpr int PROJ_THREADS = NTHREADS - 32 * KW;
 constexpr int PROJ_WARPS = PROJ_THREADS / 32;
 __device__ __forceinline__ void project_rows(const Args& a, Smem* s, int r_lo, int r_hi) {
-  const int tid = threadIdx.x - 32, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x - 32 * KW, warp = tid >> 5, lane = tid & 31;
   const int g8 = a.D / 8;
   for (int rg = r_lo; rg < r_hi; rg += RMAX) {
     const int nr = min(RMAX, r_hi - rg);
@@ -360,9 +407,9 @@ __device__ __forceinline__ void project_rows(const Args& a, Smem* s, int r_lo, i
 
 // Warp 0: ids of the keep words [dw0, dw1) (at most CHUNK_WORDS, planned in s->tab).
 // `carry` = kept blocks of the chunk's first sequence in words before dw0; returns the
-// same for the next chunk.
+// same for the next chunk. The chunk's first `own_n` words are read from s->own.
 __device__ __forceinline__ int compact_chunk(const Args& a, Smem* s, long long dw0, long long dw1,
-                                             int carry, int lane) {
+                                             int carry, int own_n, int lane) {
   const int nwc = static_cast<int>(dw1 - dw0);
   int i = 0, b = 0, wi = 0, ts = 0;
   uint32_t bits = 0;
@@ -372,7 +419,7 @@ __device__ __forceinline__ int compact_chunk(const Args& a, Smem* s, long long d
     b = s->tab.b[i];
     wi = static_cast<int>(w - s->tab.w0[i]);
     ts = s->tab.w0[i] > dw0 ? static_cast<int>(s->tab.w0[i] - dw0) : 0;  // lane of its 1st word
-    bits = __ldcg(a.words + static_cast<long long>(b) * a.n_words + wi);
+    bits = lane < own_n ? s->own[lane] : __ldcg(a.words + static_cast<long long>(b) * a.n_words + wi);
   }
   const int cnt = __popc(bits);
   int incl = cnt;
@@ -421,48 +468,56 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
     s->tab.resume_base = 0;
   }
   __syncthreads();
-  // ---- phase A. Warp 0: this CTA's keep words [W0, W1), whose first chunk of K_idx
-  // loads goes out at once; warps 1..: this CTA's rows of q.
-  if (warp == 0) {
-    const long long NW = warp_total_words(a, lane);
+  // ---- phase A. Warp 0 plans this CTA's keep words [W0, W1), and the KW copy warps
+  // start the first chunk's K_idx copies at once; warps KW..: this CTA's rows of q.
+  const long long ccap = CHUNK_WORDS / a.lk;   // words whose key rows fit in kbuf
+  if (warp < KW) {
+    if (warp == 0) {
+      SeqHead head;
+      const long long NW = warp_total_words(a, lane, head);
+      const long long W0 = (cta * NW) / G, W1 = ((cta + 1) * NW) / G;
+      if (W1 > W0) plan_chunk(a, s, W0, W1 < W0 + ccap ? W1 : W0 + ccap, lane, &head);
+      if (lane == 0) s->nw_total = NW;
+    }
+    named_bar_sync(2, KW * 32);
+    const long long NW = s->nw_total;
     const long long W0 = (cta * NW) / G, W1 = ((cta + 1) * NW) / G;
-    const long long cap = CHUNK_WORDS / a.lk;   // words whose key rows fit in kbuf
-    if (W1 > W0) issue_chunk(a, s, W0, W1 < W0 + cap ? W1 : W0 + cap, lane);
-    if (lane == 0) s->nw_total = NW;
+    if (W1 > W0) copy_chunk(a, s, W0, W1 < W0 + ccap ? W1 : W0 + ccap, tid);
   } else {
     const int RQ = a.L * D_I;
     project_rows(a, s, static_cast<int>((cta * RQ) / G), static_cast<int>(((cta + 1) * RQ) / G));
   }
-  grid_sync(a, s, 1);
+  grid_sync(a, s);
   const long long NW = s->nw_total;
   const long long W0 = (cta * NW) / G, W1 = ((cta + 1) * NW) / G;
 
   // ---- phase B: keep words, one warp per word
-  const long long ccap = CHUNK_WORDS / a.lk;
-  for (long long cw0 = W0; cw0 < W1; cw0 += ccap) {
+  int chunk = 0;
+  for (long long cw0 = W0; cw0 < W1; cw0 += ccap, ++chunk) {
     const long long cw1 = W1 < cw0 + ccap ? W1 : cw0 + ccap;
     if (cw0 != W0) {
       __syncthreads();                          // every warp is done with kbuf
-      if (warp == 0) issue_chunk(a, s, cw0, cw1, lane);
+      if (warp == 0) plan_chunk(a, s, cw0, cw1, lane);
       __syncthreads();                          // the chunk's plan is visible
+      if (warp < KW) copy_chunk(a, s, cw0, cw1, tid);
     }
-    if (warp == 0) cp_async_wait_all();         // the chunk's rows (issued by warp 0)
+    if (warp < KW) cp_async_wait_all();         // the chunk's rows (each copy warp's own)
     if (!s->abort) stage_queries(a, s);
     __syncthreads();
     if (s->abort) break;
     const int nwc = static_cast<int>(cw1 - cw0);
     for (int k = warp; k < nwc; k += NWARPS) {
-      if (a.lk > 1)
-        score_word<true>(a, s, k, cw0, lane);
-      else
-        score_word<false>(a, s, k, cw0, lane);
+      const uint32_t wor = a.lk > 1 ? score_word_any<true>(a, s, k, cw0, lane)
+                                    : score_word_any<false>(a, s, k, cw0, lane);
+      if (lane == 0 && chunk == 0) s->own[k] = wor;
     }
   }
-  grid_sync(a, s, 2);
+  grid_sync(a, s);
 
   // ---- phase C: ordered ids
   if (!s->abort && W1 > W0) {            // the same branch in every thread of the CTA
-    if (warp == 0) {
+    // The plan of [W0, W1) made in phase A is still in s->tab when phase B had one chunk.
+    if (warp == 0 && W1 - W0 > ccap) {
       s->tab.resume_b = 0;
       s->tab.resume_base = 0;
       plan_words(a, W0, W1 < W0 + CHUNK_WORDS ? W1 : W0 + CHUNK_WORDS, &s->tab, lane);
@@ -490,7 +545,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
           plan_words(a, dw0, dw1, &s->tab, lane);
           __syncwarp();
         }
-        carry = compact_chunk(a, s, dw0, dw1, carry, lane);
+        const int own_n = dw0 == W0 ? static_cast<int>(W1 - W0 < ccap ? W1 - W0 : ccap) : 0;
+        carry = compact_chunk(a, s, dw0, dw1, carry, own_n, lane);
         __syncwarp();
       }
     }
@@ -499,15 +555,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
   // sequences without candidates get a zero count; bad counts are reported once
   for (long long b = static_cast<long long>(cta) * NTHREADS + tid; b < a.B; b += G * NTHREADS) {
     if (seq_cand(a, static_cast<int>(b), true) == 0) a.sel_cnt[b] = 0;
-  }
-
-  // ---- departure: the last CTA out resets the barrier counters
-  __syncthreads();
-  if (tid == 0) {
-    if (atomicAdd(a.sync + 1, 1u) == static_cast<unsigned int>(G) - 1u) {
-      atomicExch(a.sync, 0u);
-      atomicExch(a.sync + 1, 0u);
-    }
   }
 }
 
@@ -518,8 +565,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
 namespace {
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace: q fp32 [L][B][d_i], keep words u32 [B][n_words], then the two grid-barrier
-// counters on their own 256-byte line (zero before the first call; left zero).
+// Workspace: the 64-bit grid-barrier counter on its own 256-byte line at the start (zero
+// before the first call; each call adds 2 x grid), then q fp32 [L][B][d_i] and the keep
+// words u32 [B][n_words]. The counter's place does not depend on the shape.
 struct IndexWsLayout {
   size_t q_off, words_off, sync_off, total;
   int n_words;
@@ -529,10 +577,10 @@ IndexWsLayout index_ws_layout(int B, int L, int max_cand) {
   IndexWsLayout s;
   s.n_words = (max_cand + 31) / 32;
   if (s.n_words < 1) s.n_words = 1;
-  s.q_off = 0;
+  s.sync_off = 0;
+  s.q_off = 256;
   s.words_off = align256(s.q_off + static_cast<size_t>(L) * B * lsa::idx::D_I * sizeof(float));
-  s.sync_off = align256(s.words_off + static_cast<size_t>(B) * s.n_words * sizeof(uint32_t));
-  s.total = s.sync_off + 256;
+  s.total = align256(s.words_off + static_cast<size_t>(B) * s.n_words * sizeof(uint32_t));
   return s;
 }
 
@@ -588,7 +636,7 @@ extern "C" lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const
   a.n_cand = n_cand;
   a.q = reinterpret_cast<float*>(base + lay.q_off);
   a.words = reinterpret_cast<uint32_t*>(base + lay.words_off);
-  a.sync = reinterpret_cast<unsigned int*>(base + lay.sync_off);
+  a.sync = reinterpret_cast<unsigned long long*>(base + lay.sync_off);
   a.sel_ids = sel_ids;
   a.sel_cnt = sel_cnt;
   a.logits = logits;

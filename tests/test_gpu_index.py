@@ -133,7 +133,8 @@ def test_many_short_sequences(cuda_ok):
     ws = torch.zeros(lsa.index_workspace_size(B, L, d_i, max_cand), dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     wb, hb, kb = bits(w_q), bits(h), bits(k_idx)
-    for _ in range(2):      # the workspace is reusable as left
+    G = min(torch.cuda.get_device_properties(dev).multi_processor_count, 1024)
+    for call in range(2):   # the workspace is reusable as left
         lsa.lsa_index(h.to(dev), w_q.to(dev), bias.to(dev), k_idx.to(dev), off.to(dev),
                       n_cand.to(torch.int32).to(dev), max_cand, sel_ids, sel_cnt, ws, err,
                       logits=logits)
@@ -148,4 +149,6 @@ def test_many_short_sequences(cuda_ok):
             got = ids[b, :int(cnt[b])].tolist()
             compare_selection(got, ref_ids, z_ref, "short b%d" % b)
             assert got == np.flatnonzero((z_gpu[:, b, :nc] > 0).any(axis=0)).tolist()
-        assert not ws[-256:].any()      # barrier counters left at zero
+        # the barrier counter (first 8 bytes) grew by two rounds of the grid per call
+        assert int(ws[:8].cpu().view(torch.int64)[0]) == 2 * G * (call + 1)
+        assert not ws[8:256].any()
