@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(THREADS) gather_delta_kernel(const DeltaArgs d
   __shared__ int s_fpre[MAX_DELTA_GRID + 1];   // free-page prefix over the CTAs' shares
   __shared__ int s_pend[MAX_DELTA_GRID];
   __shared__ int s_newpg[THREADS], s_item_b[THREADS], s_item_j[THREADS];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int G = gridDim.x, cta = blockIdx.x;
   if (tid == 0) s_abort = 0;
   int carry = 0;

@@ -8,11 +8,11 @@
 //
 // One cooperative launch, one CTA per SM, three phases split by two grid barriers:
 //
-//  A. Warp 0 plans the CTA's share of K_idx rows and four copy warps start their 16-byte
-//     asynchronous copies into shared memory (they do not depend on q); the other warps
-//     compute the CTA's share of the
-//     W_q rows: q[l][b][j] = W_q[l][j] . h[l][b] in fp32, each dot cut into four fixed
-//     parts summed in a fixed order.
+//  A. Warp 0 plans the CTA's share of K_idx rows and KW = 4 copy warps start their
+//     16-byte asynchronous copies into shared memory (they do not depend on q); the
+//     other warps compute the CTA's share of the W_q rows:
+//     q[l][b][j] = W_q[l][j] . h[l][b] in fp32, each dot cut into four fixed parts
+//     summed in a fixed order.
 //  B. Scoring. The candidate rows of every sequence are grouped in 32-row "words"; all
 //     words of the batch, in sequence order, are divided evenly over the CTAs. A warp
 //     scores one word from shared memory, one lane per row (rows padded by 16 bytes so
@@ -20,8 +20,9 @@
 //     z_l = q_l . k / sqrt(d_i) + bias, keep bit z_l > 0 (equal to sigmoid(z_l) > 0.5);
 //     one ballot per layer gives the word, OR-ed over the layers.
 //  C. Compaction. Each CTA ranks the kept bits of its words (popcounts of the earlier
-//     words of the same sequence, a block scan over its own) and writes the ascending id
-//     list; the CTA holding a sequence's last word writes its count.
+//     words of the same sequence, a warp scan over its own, kept in shared memory since
+//     phase B) and writes the ascending id list; the CTA holding a sequence's last word
+//     writes its count.
 //
 // Grid barriers use a 64-bit arrival counter in the workspace with a bounded wait. The
 // counter only grows (by 2 x grid per launch), so no CTA has to reset it on the way out.
