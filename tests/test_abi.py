@@ -61,6 +61,21 @@ def test_workspace_sizes(lib):
     assert lib.lsa_index_workspace_size(1, 3, 64, 100) == 0
 
 
+def test_index_workspace_layout(lib):
+    """The grid-barrier counter's 256-byte line comes first, then q fp32 [L][B][128] and
+    the keep words u32 [B][ceil(max_cand/32)], each rounded up to 256 bytes: a workspace
+    sized for one shape serves every shape that is no larger."""
+    def expect(B, L, mc):
+        r = lambda x: (x + 255) // 256 * 256
+        return 256 + r(L * B * 128 * 4) + r(B * max(1, (mc + 31) // 32) * 4)
+    for B, L, mc in ((1, 3, 16256), (64, 3, 4032), (300, 4, 90), (1, 1, 0), (7, 2, 33)):
+        assert lib.lsa_index_workspace_size(B, L, 128, mc) == expect(B, L, mc)
+    sizes = [lib.lsa_index_workspace_size(B, L, 128, mc)
+             for B in (1, 2, 9) for L in (1, 3, 4) for mc in (0, 31, 32, 1000)]
+    big = lib.lsa_index_workspace_size(9, 4, 128, 1000)
+    assert max(sizes) == big
+
+
 def test_invalid_arguments_rejected_before_device_work(lib):
     # null pointers
     assert lib.lsa_decode_attn(None, None, 1, None, 1, None, None, 1, 8, 128, 0.1, None, None, 0,
