@@ -41,7 +41,7 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "1m_b20"
 FALLBACK_HBM_GBS = 6650.0
 LAUNCHES_PER_DECODE_STEP = 1      # one fused kernel: append + split-K attention + merge
-LAUNCHES_PER_PASS_HEAD = 4        # pass set-up, projection, scoring, gather
+LAUNCHES_PER_PASS_HEAD = 3        # pass set-up, indexer (one fused launch), gather
 SEL_PAGES_CAP = 65536             # HBM pages for kept blocks at most (8 GB at d = 512)
 
 
