@@ -233,8 +233,13 @@ size_t lsa_decode_attn_workspace_size(int32_t B, int32_t H, int32_t d, int32_t n
  *  - Limit: lsa_decode_attn_workspace_size(B, H, d, n_sm) must not exceed
  *    LSA_NOALLOC_SCRATCH_BYTES (e.g. B <= 107 at H = 64, d = 512, 148 SMs); larger
  *    problems return LSA_ERR_CAPACITY before anything is enqueued.
- *  - The first call on a device looks up the array's device address and zeroes it
- *    (synchronously); make that first call before any stream capture.
+ *  - The first call on a device looks up the array's device address and enqueues, on
+ *    the caller's stream and ahead of the kernel, a clear of the array's first 256
+ *    bytes (the merge barrier counters; the partials are always written before they
+ *    are read). Make that first call before any stream capture.
+ *  - Every call leaves the counters at zero. A call whose kernel reports
+ *    LSA_DEVERR_TIMEOUT may leave them non-zero; later calls in the process are then
+ *    unreliable.
  *  - Every call shares the array: calls that overlap on the GPU (other streams,
  *    other host threads) race and produce wrong results. Serialise them.
  *  - The caller still provides and owns q, the pool, the block table, out and err.

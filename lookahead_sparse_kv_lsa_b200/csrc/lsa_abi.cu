@@ -23,6 +23,32 @@ int sm_count() {
   return cached[dev];
 }
 
+lsa_status ensure_smem_limit(const void* func, int bytes) {
+  struct Entry {
+    int dev;
+    const void* func;
+    int bytes;
+  };
+  static std::mutex mu;
+  static Entry done[256];
+  static int n_done = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].dev == dev && done[i].func == func && done[i].bytes >= bytes) return LSA_OK;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
+  if (n_done < 256) done[n_done++] = Entry{dev, func, bytes};
+  return LSA_OK;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,

@@ -28,6 +28,7 @@
 
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 
 namespace lsa {
@@ -1106,20 +1107,25 @@ size_t attn_ws_bytes(int B, int H, int d, int n_sm) {
   return (body + 255) / 256 * 256 + 256;
 }
 
+// Per-device launch state of one kernel instantiation: whether the device accepts a
+// cooperative launch that is also a programmatic dependent. Kept per device (a process
+// may drive several GPUs from several host threads).
+struct LaunchState {
+  std::atomic<int> pdl{1};        // 0: this device refused PDL with a cooperative launch
+};
+constexpr int MAX_DEVICES = 64;
+
 template <int HP, int NDC>
 lsa_status launch_attn(const CUtensorMap& mkv, const CUtensorMap& mq, const Args& a, int G,
                        cudaStream_t stream) {
   using LY = lsa::attn::Layout<HP, NDC>;
   auto kern = lsa::attn::attn_splitk_kernel<HP, NDC>;
-  static int configured_device = -1;  // the attribute is per device and function
+  static LaunchState state[MAX_DEVICES];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LSA_ERR_CUDA;
-  if (configured_device != dev) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM) !=
-        cudaSuccess)
-      return LSA_ERR_CUDA;
-    configured_device = dev;
-  }
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return LSA_ERR_CUDA;
+  LaunchState& ls = state[dev];
+  const lsa_status st = lsa_host::ensure_smem_limit(reinterpret_cast<const void*>(kern), LY::SMEM);
+  if (st != LSA_OK) return st;
   // Cooperative launch: all G CTAs (one per SM) are resident together, which the
   // fused merge's grid barrier relies on.
   cudaLaunchConfig_t cfg = {};
@@ -1129,18 +1135,21 @@ lsa_status launch_attn(const CUtensorMap& mkv, const CUtensorMap& mq, const Args
   cfg.stream = stream;
   // Programmatic stream serialisation lets this launch's CTAs set up while the previous
   // kernel in the stream drains; the kernel waits for it before touching any data.
-  static bool pdl_ok = true;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_ok ? 2 : 1;
-  if (cudaLaunchKernelEx(&cfg, kern, mkv, mq, a) == cudaSuccess) return LSA_OK;
+  const bool pdl = ls.pdl.load(std::memory_order_relaxed) != 0;
+  cfg.numAttrs = pdl ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mkv, mq, a);
+  if (e == cudaSuccess) return LSA_OK;
   cudaGetLastError();
-  if (!pdl_ok) return LSA_ERR_CUDA;
-  pdl_ok = false;  // this driver refuses the combination: plain cooperative launches
+  // Only the answer "not supported" to the attribute combination turns PDL off (for this
+  // device, for good); any other failure is reported to the caller as it is.
+  if (!pdl || e != cudaErrorNotSupported) return LSA_ERR_CUDA;
+  ls.pdl.store(0, std::memory_order_relaxed);
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, mkv, mq, a) != cudaSuccess) {
     cudaGetLastError();
@@ -1165,13 +1174,13 @@ lsa_status dispatch_d(const CUtensorMap& mkv, const CUtensorMap& mq, const Args&
 
 namespace lsa_host {
 
-lsa_status decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pages,
-                       const int32_t* block_table, int32_t bt_stride, const int32_t* n_entries,
-                       const int32_t* tail_len, int32_t B, int32_t H, int32_t d, float scale,
-                       uint16_t* out, void* ws, size_t ws_bytes, int32_t* err, void* stream,
-                       const AppendArgs* append) {
-  if (!q || !hbm_pool || !block_table || !n_entries || !out || !ws || !err)
-    return LSA_ERR_INVALID_ARG;
+// Host checks of every argument of a decode-attention call except the workspace.
+lsa_status check_attn_args(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pages,
+                           const int32_t* block_table, int32_t bt_stride,
+                           const int32_t* n_entries, const int32_t* tail_len, int32_t B,
+                           int32_t H, int32_t d, float scale, const uint16_t* out,
+                           const int32_t* err, const AppendArgs* append) {
+  if (!q || !hbm_pool || !block_table || !n_entries || !out || !err) return LSA_ERR_INVALID_ARG;
   if (!append && !tail_len) return LSA_ERR_INVALID_ARG;
   if (append && (!append->k_new || !append->v_new || append->tail < 1 || append->tail > 64))
     return LSA_ERR_INVALID_ARG;
@@ -1181,12 +1190,24 @@ lsa_status decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pa
   if (n_pages > (int64_t(1) << 23)) return LSA_ERR_INVALID_ARG;  // page rows must fit in int32
   if (static_cast<int64_t>(B) * H > (int64_t(1) << 30)) return LSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(hbm_pool) |
-       reinterpret_cast<uintptr_t>(ws)) & 15u)
+       reinterpret_cast<uintptr_t>(out)) & 15u)
     return LSA_ERR_INVALID_ARG;
   if (append && ((reinterpret_cast<uintptr_t>(append->k_new) |
                   reinterpret_cast<uintptr_t>(append->v_new)) & 15u))
     return LSA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(out) & 15u) != 0) return LSA_ERR_INVALID_ARG;
+  return LSA_OK;
+}
+
+lsa_status decode_attn(const uint16_t* q, const uint16_t* hbm_pool, int64_t n_pages,
+                       const int32_t* block_table, int32_t bt_stride, const int32_t* n_entries,
+                       const int32_t* tail_len, int32_t B, int32_t H, int32_t d, float scale,
+                       uint16_t* out, void* ws, size_t ws_bytes, int32_t* err, void* stream,
+                       const AppendArgs* append) {
+  lsa_host::NvtxRange nvtx_range("lsa_decode_attn");
+  lsa_status st0 = check_attn_args(q, hbm_pool, n_pages, block_table, bt_stride, n_entries,
+                                   tail_len, B, H, d, scale, out, err, append);
+  if (st0 != LSA_OK) return st0;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15u)) return LSA_ERR_INVALID_ARG;
   const int G = sm_count();
   if (G <= 0) return LSA_ERR_CUDA;
   if (G > lsa::attn::MAX_GRID) return LSA_ERR_UNIMPLEMENTED;
@@ -1270,11 +1291,17 @@ std::mutex g_noalloc_mutex;
 NoallocScratch g_noalloc[64];
 
 // Device address of the scratch array on the current device. In host code the array's
-// name is only a host-side stand-in, so the address is queried once per device (with
-// that device current) and the barrier counters are zeroed then.
-lsa_status noalloc_scratch(void** out) {
+// name is only a host-side stand-in, so the address is looked up once per device, with
+// that device current. That first time, a clear of the array's first 256 bytes (the
+// merge barrier counters; partials are always written before they are read) is enqueued
+// on the caller's stream, so it is ordered before the kernel launched next on the same
+// stream. (Global device variables without an initialiser also start at zero.)
+lsa_status noalloc_scratch(void** out, cudaStream_t stream) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LSA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   NoallocScratch& s = g_noalloc[dev];
   if (!s.ready) {
@@ -1283,7 +1310,7 @@ lsa_status noalloc_scratch(void** out) {
       cudaGetLastError();
       return LSA_ERR_CUDA;
     }
-    if (cudaMemset(p, 0, LSA_NOALLOC_SCRATCH_BYTES) != cudaSuccess) {
+    if (cudaMemsetAsync(p, 0, 256, stream) != cudaSuccess) {
       cudaGetLastError();
       return LSA_ERR_CUDA;
     }
@@ -1302,13 +1329,17 @@ extern "C" lsa_status lsa_decode_attn_noalloc(const uint16_t* q, const uint16_t*
                                               const int32_t* tail_len, int32_t B, int32_t H,
                                               int32_t d, float scale, uint16_t* out,
                                               int32_t* err, void* stream) {
-  if (B <= 0 || H <= 0 || d <= 0) return LSA_ERR_INVALID_ARG;
+  // the arguments first, so that a malformed call is told so and not that it is too big
+  const lsa_status chk = lsa_host::check_attn_args(q, hbm_pool, n_pages, block_table, bt_stride,
+                                                   n_entries, tail_len, B, H, d, scale, out, err,
+                                                   nullptr);
+  if (chk != LSA_OK) return chk;
   const int G = lsa_host::sm_count();
   if (G <= 0) return LSA_ERR_CUDA;
   const size_t need = attn_ws_bytes(B, H, d, G);
   if (need > static_cast<size_t>(LSA_NOALLOC_SCRATCH_BYTES)) return LSA_ERR_CAPACITY;
   void* ws = nullptr;
-  const lsa_status st = noalloc_scratch(&ws);
+  const lsa_status st = noalloc_scratch(&ws, static_cast<cudaStream_t>(stream));
   if (st != LSA_OK) return st;
   return lsa_host::decode_attn(q, hbm_pool, n_pages, block_table, bt_stride, n_entries, tail_len,
                                B, H, d, scale, out, ws, need, err, stream, nullptr);

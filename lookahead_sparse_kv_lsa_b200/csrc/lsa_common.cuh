@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/lsa.h"
 
@@ -331,10 +332,23 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t byte_in_
 // ------------------------------------------------------------------- host helpers
 namespace lsa_host {
 
+// Names the host-side enqueue of one library call in profiler timelines (NVTX; a no-op
+// unless a profiling tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 inline lsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA; }
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
+
+// Raise the dynamic shared-memory limit of `func` to `bytes` on the current device,
+// once per (device, function); later calls return at once. Thread-safe.
+lsa_status ensure_smem_limit(const void* func, int bytes);
 
 // cuTensorMapEncodeTiled, fetched through the runtime so the library does not link
 // against libcuda (it loads on machines without a driver).

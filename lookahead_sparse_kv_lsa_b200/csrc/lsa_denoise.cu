@@ -766,6 +766,7 @@ extern "C" lsa_status lsa_denoise_labels(const float* logits, int32_t n_windows,
                                          int32_t* set_cnt, uint32_t* label_mask,
                                          int32_t* label_ids, int32_t label_cap,
                                          int32_t* label_cnt, int32_t* err, void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_denoise_labels");
   using namespace lsa;
   if (logits == nullptr || set_mask == nullptr || label_cnt == nullptr) return LSA_ERR_INVALID_ARG;
   if (n_windows < 1 || n_layers < 1 || n_layers >= (1 << DN_PLANES) || n_blocks < 1 ||
@@ -774,16 +775,14 @@ extern "C" lsa_status lsa_denoise_labels(const float* logits, int32_t n_windows,
   if (static_cast<int64_t>(n_windows) * n_layers > 0x7fffffffLL) return LSA_ERR_INVALID_ARG;
   if (!(top_p > 0.0) || !(top_p <= 1.0)) return LSA_ERR_INVALID_ARG;
   if (label_cap < 0 || (label_cap > 0 && label_ids == nullptr)) return LSA_ERR_INVALID_ARG;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(denoise_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem_bytes(LSA_DENOISE_MAX_BLOCKS / 32))) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(vote_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(vote_smem_bytes(LSA_DENOISE_MAX_BLOCKS / 32))) !=
-            cudaSuccess)
-      return LSA_ERR_CUDA;
-    attr = true;
+  {
+    lsa_status st = lsa_host::ensure_smem_limit(
+        reinterpret_cast<const void*>(denoise_kernel),
+        static_cast<int>(smem_bytes(LSA_DENOISE_MAX_BLOCKS / 32)));
+    if (st == LSA_OK)
+      st = lsa_host::ensure_smem_limit(reinterpret_cast<const void*>(vote_kernel),
+                                       static_cast<int>(vote_smem_bytes(LSA_DENOISE_MAX_BLOCKS / 32)));
+    if (st != LSA_OK) return st;
   }
   DenoiseArgs a{};
   a.logits = logits;

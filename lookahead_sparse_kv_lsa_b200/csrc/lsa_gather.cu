@@ -511,6 +511,7 @@ extern "C" lsa_status lsa_gather(const uint16_t* host_pool, int64_t host_blocks,
                                  uint16_t* hbm_pool, int64_t n_pages, int32_t sel_page_base,
                                  int32_t sel_page_count, int32_t* block_table, int32_t bt_stride,
                                  int32_t* n_entries, int32_t* err, void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_gather");
   if (!host_pool || !host_blk_off || !sel_cnt || !res_pages || !n_res || !hbm_pool ||
       !block_table || !n_entries || !err)
     return LSA_ERR_INVALID_ARG;
@@ -585,6 +586,7 @@ extern "C" lsa_status lsa_gather_delta(
     int64_t n_pages, int32_t sel_page_base, int32_t sel_page_count, int32_t* block_table,
     int32_t bt_stride, int32_t* n_entries, int32_t* kept_ids, int32_t* kept_pages,
     int32_t* kept_cnt, void* ws, size_t ws_bytes, int32_t* copied, int32_t* err, void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_gather_delta");
   if (!host_pool || !host_blk_off || !sel_cnt || !res_pages || !n_res || !hbm_pool ||
       !block_table || !n_entries || !err || !kept_cnt || !ws)
     return LSA_ERR_INVALID_ARG;
@@ -675,6 +677,7 @@ lsa::gth::StepArgs step_args(const lsa_state* st, const void* host_dev) {
 }  // namespace
 
 extern "C" lsa_status lsa_load_window(const lsa_state* st, int32_t pass, void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_load_window");
   const lsa_status v = lsa_state_check(st);
   if (v != LSA_OK) return v;
   if (pass < 0) return LSA_ERR_INVALID_ARG;
@@ -688,6 +691,7 @@ extern "C" lsa_status lsa_load_window(const lsa_state* st, int32_t pass, void* s
 }
 
 extern "C" lsa_status lsa_pass_setup(const lsa_state* st, int32_t pass, void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_pass_setup");
   const lsa_status v = lsa_state_check(st);
   if (v != LSA_OK) return v;
   if (pass < 0) return LSA_ERR_INVALID_ARG;
@@ -700,6 +704,7 @@ extern "C" lsa_status lsa_pass_setup(const lsa_state* st, int32_t pass, void* st
 
 extern "C" lsa_status lsa_append(const lsa_state* st, int64_t step, const uint16_t* k_new,
                                  const uint16_t* v_new, void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_append");
   const lsa_status v = lsa_state_check(st);
   if (v != LSA_OK) return v;
   if (step < 0 || step / LSA_TAU > (int64_t(1) << 30) || !k_new || !v_new)
@@ -734,6 +739,7 @@ extern "C" lsa_status lsa_decode_step(const lsa_state* st, int64_t step, const u
 extern "C" lsa_status lsa_step(const lsa_state* st, int64_t step, const uint16_t* h,
                                const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
                                uint16_t* out, void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_step");
   lsa_status v = lsa_state_check(st);
   if (v != LSA_OK) return v;
   if (step < 0 || step / LSA_TAU > (int64_t(1) << 30) || !q || !k_new || !v_new || !out)

@@ -600,6 +600,7 @@ extern "C" lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const
                                    int32_t* sel_ids, int32_t* sel_cnt, int32_t cap, float* logits,
                                    uint32_t* layer_mask, void* ws, size_t ws_bytes, int32_t* err,
                                    void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_index");
   if (!h || !w_q || !bias || !k_idx || !kidx_off || !n_cand || !sel_cnt || !ws || !err)
     return LSA_ERR_INVALID_ARG;
   if (kidx_layer_stride < 0) return LSA_ERR_INVALID_ARG;
@@ -616,14 +617,10 @@ extern "C" lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const
   if (n_sm <= 0) return LSA_ERR_CUDA;
   const int G = n_sm < lsa::idx::MAX_GRID ? n_sm : lsa::idx::MAX_GRID;
 
-  static int configured_device = -1;   // the attribute is per device and function
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LSA_ERR_CUDA;
-  if (configured_device != dev) {
-    if (cudaFuncSetAttribute(lsa::idx::index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kIndexSmem)) != cudaSuccess)
-      return LSA_ERR_CUDA;
-    configured_device = dev;
+  {
+    const lsa_status st = lsa_host::ensure_smem_limit(
+        reinterpret_cast<const void*>(lsa::idx::index_kernel), static_cast<int>(kIndexSmem));
+    if (st != LSA_OK) return st;
   }
   uint8_t* base = static_cast<uint8_t*>(ws);
   lsa::idx::Args a;

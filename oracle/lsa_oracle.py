@@ -23,7 +23,7 @@ Lookahead Sparse Attention" (zhichai.net), section 2 "Core Idea of LSA", steps 1
      window and the tokens decoded since the pass started);
   5. after 64 steps the indexer runs again.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
   * blocks are 64 tokens; the recent window W is part of the workload;
   * only blocks that end before the window are candidates;
   * the window grows with the decoded tokens inside a pass and is re-based at the

@@ -43,3 +43,25 @@ def compare_selection(gpu_ids, ref_ids, ref_z, what=""):
 
 def bits(t: torch.Tensor) -> np.ndarray:
     return bf16_bits(t.cpu() if t.is_cuda else t)
+
+
+def paged_oracle_out(pool, bt, q, entries, tails, scale):
+    """The oracle's attention over paged KV: sequence b attends to the tokens of pages
+    bt[b][0 .. entries[b]-1], all 64 tokens of each except tails[b] of the last one.
+    Returns float64 [B][H][d] (zero for a sequence without pages)."""
+    B, H, d = q.shape
+    pb = bits(pool)
+    out = np.zeros((B, H, d))
+    for b in range(B):
+        if entries[b] == 0:
+            continue
+        Ks, Vs = [], []
+        for e in range(entries[b]):
+            page = int(bt[b, e])
+            n = 64 if e < entries[b] - 1 else tails[b]
+            Ks.append(pb[page, 0, :n])
+            Vs.append(pb[page, 1, :n])
+        K = oracle.bf16_to_f64(np.concatenate(Ks))
+        V = oracle.bf16_to_f64(np.concatenate(Vs))
+        out[b] = oracle.softmax_attention(oracle.bf16_to_f64(bits(q[b])), K, V, scale)
+    return out

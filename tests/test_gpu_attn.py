@@ -9,7 +9,7 @@ import torch
 
 import lookahead_sparse_kv_lsa_b200 as lsa
 import oracle
-from gpu_util import compare_attention, bits
+from gpu_util import compare_attention, bits, paged_oracle_out
 
 pytestmark = pytest.mark.gpu
 
@@ -34,21 +34,7 @@ def make_case(seed, B, H, d, entries, tails, n_pages=None, q_scale=1.0, garbage=
     return pool, bt, q
 
 
-def oracle_out(pool, bt, q, entries, tails, scale):
-    B, H, d = q.shape
-    pb = bits(pool)
-    out = np.zeros((B, H, d))
-    for b in range(B):
-        if entries[b] == 0:
-            continue
-        Ks, Vs = [], []
-        for e in range(entries[b]):
-            page = int(bt[b, e])
-            n = 64 if e < entries[b] - 1 else tails[b]
-            Ks.append(pb[page, 0, :n]); Vs.append(pb[page, 1, :n])
-        K = oracle.bf16_to_f64(np.concatenate(Ks)); V = oracle.bf16_to_f64(np.concatenate(Vs))
-        out[b] = oracle.softmax_attention(oracle.bf16_to_f64(bits(q[b])), K, V, scale)
-    return out
+oracle_out = paged_oracle_out
 
 
 def run_gpu(pool, bt, q, entries, tails, scale):
