@@ -468,29 +468,34 @@ def barrier(world):
 
 def e2e_measure(dec, wl, dev, passes, world, total_seqs=None):
     """Throughput through lsa_step from Python with host buffers: each decode step copies
-    its inputs host->device (and h at the pass start) and reads its output back."""
+    its inputs host->device in one copy (q, k_new and v_new packed in one pinned staging
+    row; h joins the row at the pass start) and reads its output back in one copy."""
     import torch
     import lookahead_sparse_kv_lsa_b200 as lsa
     c = wl.cfg
-    h_host = wl.h(0).pin_memory()
-    q_host = torch.stack([wl.q(0, s) for s in range(c.tau)]).pin_memory()
-    kv = [wl.kv_new(0, s) for s in range(c.tau)]
-    k_host = torch.stack([a for a, _ in kv]).pin_memory()
-    v_host = torch.stack([b for _, b in kv]).pin_memory()
+    nq, nk, nh = c.B * c.H * c.d, c.B * c.d, c.L * c.B * c.D
+    row = nq + 2 * nk
+    # per step: [q | k_new | v_new], and h after them in step 0's row (bf16 elements;
+    # every piece starts on a 16-byte boundary)
+    host = torch.empty((c.tau, row + nh), dtype=torch.bfloat16).pin_memory()
+    for s in range(c.tau):
+        k, v = wl.kv_new(0, s)
+        host[s, :nq] = wl.q(0, s).reshape(-1)
+        host[s, nq:nq + nk] = k.reshape(-1)
+        host[s, nq + nk:row] = v.reshape(-1)
+    host[0, row:] = wl.h(0).reshape(-1)
     out_host = torch.empty((c.tau, c.B, c.H, c.d), dtype=torch.bfloat16).pin_memory()
-    h_d = torch.empty_like(h_host, device=dev)
-    q_d = torch.empty((c.B, c.H, c.d), dtype=torch.bfloat16, device=dev)
-    k_d = torch.empty((c.B, c.d), dtype=torch.bfloat16, device=dev)
-    v_d = torch.empty_like(k_d)
-    o_d = torch.empty_like(q_d)
+    stage = torch.empty(row + nh, dtype=torch.bfloat16, device=dev)
+    q_d = stage[:nq].view(c.B, c.H, c.d)
+    k_d = stage[nq:nq + nk].view(c.B, c.d)
+    v_d = stage[nq + nk:row].view(c.B, c.d)
+    h_d = stage[row:].view(c.L, c.B, c.D)
+    o_d = torch.empty((c.B, c.H, c.d), dtype=torch.bfloat16, device=dev)
 
     def one_pass():
         for s in range(c.tau):
-            if s == 0:
-                h_d.copy_(h_host, non_blocking=True)
-            q_d.copy_(q_host[s], non_blocking=True)
-            k_d.copy_(k_host[s], non_blocking=True)
-            v_d.copy_(v_host[s], non_blocking=True)
+            n = row + nh if s == 0 else row
+            stage[:n].copy_(host[s, :n], non_blocking=True)
             lsa.lsa_step(dec.state, s, h_d if s == 0 else None, q_d, k_d, v_d, o_d)
             out_host[s].copy_(o_d, non_blocking=True)
 
@@ -505,11 +510,12 @@ def e2e_measure(dec, wl, dev, passes, world, total_seqs=None):
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), world)
     barrier(world)
-    h2d = h_host.numel() * 2 + c.tau * (q_host[0].numel() + 2 * k_host[0].numel()) * 2
+    h2d = 2 * (nh + c.tau * row)
     d2h = c.tau * out_host[0].numel() * 2
     seqs = total_seqs if total_seqs is not None else world * c.B
     return {"value": seqs * c.tau * passes / (ms * 1e-3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "copies_per_decode_step": {"h2d": 1, "d2h": 1},
             "ms_per_step": ms / passes, "api": "lsa_step (Python ctypes), pinned host buffers"}
 
 
@@ -610,6 +616,50 @@ def denoise_report(dev, hbm, with_oracle=True, reps=20):
     del copies
     torch.cuda.empty_cache()
     return res
+
+
+def near_tie_band(wl, dec, dev, band=1e-3):
+    """Blocks whose logit lies within `band` of the threshold in some indexer layer, from
+    the kernel's own logits (one extra lsa_index call after the timed region). The block
+    selection may legitimately differ from an exact computation only on such blocks."""
+    import torch
+    import lookahead_sparse_kv_lsa_b200 as lsa
+    c = wl.cfg
+    mc = dec.max_cand
+    logits = torch.full((c.L, c.B, mc), float("inf"), device=dev)
+    ids = torch.empty_like(dec.sel_ids)
+    cnt = torch.empty_like(dec.sel_cnt)
+    h = wl.h(0).to(dev)
+    lsa.lsa_index(h, dec.w_q, dec.bias, dec.k_idx, dec.kidx_off, dec.n_cand, mc, ids, cnt,
+                  dec.index_ws, dec.err, logits=logits)
+    torch.cuda.synchronize()
+    z = logits.abs().amin(dim=0)                      # [B][max_cand]; inf past n_cand
+    per_seq = (z < band).sum(dim=1).cpu().tolist()
+    return {"band": band, "blocks_in_band": int(sum(per_seq)),
+            "candidates": int(dec.n_cand.sum()), "source": "kernel logits"}
+
+
+def oracle_flips(wl, dec):
+    """Selection differences against the oracle for the sampled sequences of pass 0:
+    blocks selected by one side only, all of which must lie in the near-tie band."""
+    import numpy as np
+    import oracle
+    from lsa_inputs import bf16_bits
+    c = wl.cfg
+    hb = bf16_bits(wl.h(0))
+    wq = bf16_bits(wl.w_q)
+    flips, in_band = 0, 0
+    seqs = sample_sequences(c.B)
+    for b in seqs:
+        nc = oracle.n_candidates(int(wl.ctx_at(0)[b]), c.W)
+        kb = wl.seq_k_idx(b)
+        kb = kb[:, :nc] if kb.dim() == 3 else kb[:nc]
+        ref, z = oracle.index_pass(wq, hb[:, b], bf16_bits(kb), float(wl.bias[b]))
+        got = set(dec.sel_ids[b, :int(dec.sel_cnt[b])].cpu().tolist())
+        diff = got ^ set(int(x) for x in ref)
+        flips += len(diff)
+        in_band += sum(1 for x in diff if float(np.min(np.abs(z[:, x]))) < 1e-3)
+    return {"sequences": seqs, "flipped_blocks": flips, "flipped_in_band": in_band}
 
 
 def spot_check(wl, out, dec):
@@ -733,7 +783,7 @@ def run_lsa(args, rank, world, local):
         "gpu_launches": args.steps * (LAUNCHES_PER_PASS_HEAD + cfg.tau * LAUNCHES_PER_DECODE_STEP),
         "clocks": clocks,
     }
-    line["parity_spot_check_max_abs"] = spot_check(wl, out, dec) if rank == 0 else None
+    line["near_ties"] = near_tie_band(wl, dec, dev)
     del graphs, events
     if not args.no_dense and cfg.B == 1:
         dms, dbytes, dT = dense_attention(wl, dec, dev)
@@ -750,6 +800,9 @@ def run_lsa(args, rank, world, local):
         # the default workload samples all 64 steps; the others four of them
         steps = tuple(range(cfg.tau)) if cfg.name == DEFAULT_WORKLOAD else (0, 21, 42, 63)
         line["cpu_baseline"] = cpu_baseline(wl, steps)
+        # the oracle leg also checks the timed run's last step and selection
+        line["parity_spot_check_max_abs"] = spot_check(wl, out, dec)
+        line["near_ties"]["oracle"] = oracle_flips(wl, dec)
     if cfg.passes > 1:
         line["delta_gather"] = delta_gather_report(wl, dev)
     if rank == 0 and world == 1 and not args.no_denoise:

@@ -150,6 +150,28 @@ def softmax_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float)
     return (p @ V) / p.sum(axis=1, keepdims=True)
 
 
+def softmax_attention_bits(q: np.ndarray, K_bits, V_bits, scale: float,
+                           chunk: int = 65536) -> np.ndarray:
+    """softmax_attention over keys and values given as bf16 bit patterns [T][d], decoded
+    a chunk of rows at a time, so that a context of a million tokens fits in memory.
+
+    Two passes: every score scale * q_h . K_t (float64), then the exact softmax weights
+    exp(score - max) applied to V chunk by chunk. Equal to softmax_attention on the
+    decoded arrays up to the order of the float64 sums.
+    """
+    T = K_bits.shape[0]
+    if T == 0:
+        return np.zeros((q.shape[0], V_bits.shape[1]))
+    scores = np.empty((q.shape[0], T))
+    for t0 in range(0, T, chunk):
+        scores[:, t0:t0 + chunk] = scale * (q @ bf16_to_f64(K_bits[t0:t0 + chunk]).T)
+    p = np.exp(scores - scores.max(axis=1, keepdims=True))
+    out = np.zeros((q.shape[0], V_bits.shape[1]))
+    for t0 in range(0, T, chunk):
+        out += p[:, t0:t0 + chunk] @ bf16_to_f64(V_bits[t0:t0 + chunk])
+    return out / p.sum(axis=1, keepdims=True)
+
+
 def step_output(q_bits, K_bits, V_bits, ids, n_ctx: int, window: int, s: int, scale: float,
                 heads: Optional[Sequence[int]] = None, block: int = BLOCK) -> np.ndarray:
     """Attention output of one decode step of one sequence, float64 [H'][d].

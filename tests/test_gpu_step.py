@@ -47,9 +47,14 @@ def run_loop(wl, keep_steps):
     return outs, sels
 
 
-def check_loop(wl, keep_steps, heads=None):
+def check_loop(wl, keep_steps, heads=None, seqs=None):
+    """Selection of every sequence in every pass against the oracle (exact outside the
+    near-tie band); attention of the sequences `seqs` (all by default) on the kept steps
+    and heads. Returns the near-tie flips per pass."""
     c = wl.cfg
     outs, sels = run_loop(wl, keep_steps)
+    check_b = set(range(c.B)) if seqs is None else set(seqs)
+    flips = []
     wq = bits(wl.w_q)
     for p in range(c.passes):
         hb = bits(wl.h(p))
@@ -62,6 +67,9 @@ def check_loop(wl, keep_steps, heads=None):
             ref_ids, z = oracle.index_pass(wq, hb[:, b], bits(kb), float(wl.bias[b]))
             got = ids_gpu[b, :int(cnt_gpu[b])].tolist()
             near = compare_selection(got, ref_ids, z, "%s p%d b%d" % (c.name, p, b))
+            flips.append(len(near))
+            if b not in check_b:
+                continue
             # with near-tie flips, attention is checked over the GPU's own selection
             use_ids = got if near else ref_ids
             K, V = wl.seq_kv(b)
@@ -73,6 +81,8 @@ def check_loop(wl, keep_steps, heads=None):
                 if heads is not None:
                     got_o = got_o[list(heads)]
                 compare_attention(got_o, ref, "%s p%d s%d b%d" % (c.name, p, s, b))
+    print("%s: near-tie flips %d over %d sequence passes" % (c.name, sum(flips), len(flips)))
+    return flips
 
 
 def test_tiny_every_step(cuda_ok):
@@ -110,3 +120,92 @@ def test_mid_batch_full_sampled(cuda_ok):
     """B=8 x 131,072 tokens: steps 0 and 63 on two sampled heads of every sequence."""
     wl = LI.Workload(LI.mid_batch(), pin=True)
     check_loop(wl, {0, 63}, heads=[5, 60])
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("bias", [-1.5, -2.5])
+def test_one_million_other_biases_full_sampled(cuda_ok, bias):
+    """1M tokens at bias -1.5 (~3,000 kept blocks, 416 MB per step) and -2.5: steps 0
+    and 63 on four heads."""
+    wl = LI.Workload(LI.one_million(bias), pin=True)
+    check_loop(wl, {0, 63}, heads=[0, 21, 42, 63])
+
+
+@pytest.mark.slow
+def test_long_context_four_passes_full_sampled(cuda_ok):
+    """B=4 x 524,288 tokens, all four indexer passes: steps 0 and 63 of every pass on two
+    heads of every sequence (the window slides and the candidates grow each pass)."""
+    wl = LI.Workload(LI.long_ctx(), pin=True)
+    check_loop(wl, {0, 63}, heads=[7, 56])
+
+
+@pytest.mark.slow
+def test_ragged_mix_full_sampled(cuda_ok):
+    """B=64 sequences of 32K..256K tokens with per-sequence bias: the selection of all 64,
+    attention of 8 sampled sequences (the shortest, the longest and six spread over the
+    batch) at steps 0 and 63 on two heads."""
+    wl = LI.Workload(LI.ragged_mix(), pin=True)
+    ctx = wl.ctx0
+    spread = [int(x) for x in np.linspace(0, wl.cfg.B - 1, 6).round()]
+    seqs = sorted(set([int(np.argmin(ctx)), int(np.argmax(ctx))] + spread))
+    check_loop(wl, {0, 63}, heads=[3, 50], seqs=seqs)
+
+
+@pytest.mark.slow
+def test_dense_one_million_full(cuda_ok):
+    """Dense decode at 1M tokens: lsa_decode_attn over every block of the context (16,385
+    pages, the last one full), with the queries of steps 0 and 63, on four heads, against
+    the oracle's softmax over all 1,048,640 tokens."""
+    dev = torch.device("cuda")
+    wl = LI.Workload(LI.one_million(-2.0), pin=True)
+    c = wl.cfg
+    n = int(wl.nb0[0]) + 1
+    pool = wl.host_pool[:n].to(dev)
+    bt = torch.arange(n, dtype=torch.int32, device=dev).view(1, n)
+    ne = torch.tensor([n], dtype=torch.int32, device=dev)
+    tl = torch.tensor([64], dtype=torch.int32, device=dev)
+    ws = torch.zeros(lsa.decode_attn_workspace_size(1, c.H, c.d), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    K, V = wl.seq_kv(0)
+    T = n * 64
+    Kb, Vb = bits(K[:T]), bits(V[:T])
+    heads = [0, 21, 42, 63]
+    for s in (0, 63):
+        q = wl.q(0, s).to(dev)
+        out = torch.full_like(q, float("nan"))
+        lsa.lsa_decode_attn(q, pool, bt, ne, tl, c.scale, out, ws, err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        qf = oracle.bf16_to_f64(bits(wl.q(0, s)[0]))[heads]
+        ref = oracle.softmax_attention_bits(qf, Kb, Vb, c.scale)
+        compare_attention(out[0][heads], ref, "dense 1M s%d" % s)
+
+
+def test_shard_is_the_same_computation(cuda_ok):
+    """A rank's shard of a batch (sequences 4..8 of a scaled-down ragged batch of 12)
+    decoded alone on one GPU equals the oracle fed from the whole batch's draws for
+    those sequences: sharding by sequence changes nothing in what is computed."""
+    full = LI.Workload(LI.scaled_down(LI.ragged_mix(), ctx_blocks=160, B=12), pin=True)
+    shard = LI.Workload(LI.scaled_down(LI.ragged_mix(), ctx_blocks=160, B=12), pin=True,
+                        seqs=range(4, 9))
+    c = shard.cfg
+    steps = {0, 31, 63}
+    outs, sels = run_loop(shard, steps)
+    wq = bits(full.w_q)
+    hb = bits(full.h(0))
+    for i, b in enumerate(range(4, 9)):
+        n_ctx = int(full.ctx_at(0)[b])
+        assert n_ctx == int(shard.ctx_at(0)[i])
+        nc = oracle.n_candidates(n_ctx, c.W)
+        ref_ids, z = oracle.index_pass(wq, hb[:, b], bits(full.seq_k_idx(b)[:nc]),
+                                       float(full.bias[b]))
+        ids_gpu, cnt_gpu = sels[0]
+        got = ids_gpu[i, :int(cnt_gpu[i])].tolist()
+        near = compare_selection(got, ref_ids, z, "shard seq %d" % b)
+        use_ids = got if near else ref_ids
+        K, V = full.seq_kv(b)
+        Kb, Vb = bits(K), bits(V)
+        for s in sorted(steps):
+            qf = bits(full.q(0, s)[b])
+            ref = oracle.step_output(qf, Kb, Vb, use_ids, n_ctx, c.W, s, c.scale)
+            compare_attention(outs[(0, s)][i], ref, "shard seq %d s%d" % (b, s))

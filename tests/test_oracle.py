@@ -156,6 +156,23 @@ def check_matches_sdpa(O=O):
     assert np.max(np.abs(out - ref)) < 1e-12
 
 
+def check_chunked_attention_matches_whole(O=O):
+    """The chunked form over bf16 bits equals the whole-array form, for chunk sizes that
+    do and do not divide T, and for a chunk larger than T."""
+    rng = np.random.default_rng(11)
+    H, T, d = 4, 1000, 32
+    K_bits = f64_to_bf16_bits(np.round(rng.standard_normal((T, d)) * 8) / 8)
+    V_bits = f64_to_bf16_bits(np.round(rng.standard_normal((T, d)) * 8) / 8)
+    q = rng.standard_normal((H, d))
+    whole = O.softmax_attention(q, O.bf16_to_f64(K_bits), O.bf16_to_f64(V_bits), 0.25)
+    for chunk in (1, 7, 128, 1000, 4096):
+        got = O.softmax_attention_bits(q, K_bits, V_bits, 0.25, chunk=chunk)
+        assert np.max(np.abs(got - whole)) < 1e-12, chunk
+    # one token: exactly that token's V for every head
+    one = O.softmax_attention_bits(q, K_bits[:1], V_bits[:1], 0.25, chunk=1)
+    assert np.array_equal(one, np.repeat(O.bf16_to_f64(V_bits[:1]), H, axis=0))
+
+
 def check_uniform_when_q_zero(O=O):
     rng = np.random.default_rng(7)
     K = rng.standard_normal((50, 16)); V = rng.standard_normal((50, 16))
@@ -314,7 +331,7 @@ def check_vote(O=O):
 PINS = [check_bf16_decode, check_projection_unit_rows, check_projection_bruteforce,
         check_logits_closed_form, check_per_layer_keys, check_threshold_strict, check_union_bruteforce,
         check_selection_rate, check_single_token, check_two_token_closed_form,
-        check_matches_sdpa, check_uniform_when_q_zero, check_attended_set,
+        check_matches_sdpa, check_chunked_attention_matches_whole, check_uniform_when_q_zero, check_attended_set,
         check_special_cases_reduce_to_dense, check_top_p_closed_forms, check_top_p_bruteforce,
         check_vote]
 
@@ -419,6 +436,10 @@ MUTANTS = {
     "top_p_ties_by_high_id": dict(top_p_set=lambda pr, p: _top_p_variant(pr, p, high_id=True)),
     "top_p_one_extra": dict(top_p_set=lambda pr, p: _top_p_variant(pr, p, extra=1)),
     "vote_ge_2": dict(denoise_labels=lambda lg, p=0.6, min_votes=3: O.denoise_labels(lg, p, 2)),
+    "chunked_attention_drops_ragged_tail": dict(
+        softmax_attention_bits=lambda q, Kb, Vb, sc, chunk=65536: O.softmax_attention_bits(
+            q, Kb[:max(chunk, len(Kb) // chunk * chunk)], Vb[:max(chunk, len(Kb) // chunk * chunk)],
+            sc, chunk)),
     "bf16_truncated_wrong_shift": dict(bf16_to_f64=lambda b: (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(15)).view(np.float32).astype(np.float64)),
 }
 
