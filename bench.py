@@ -57,6 +57,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-denoise", action="store_true",
                     help="skip the label-denoising report (64 windows x 21 layers x 16,384 blocks)")
+    ap.add_argument("--no-lowrank", action="store_true",
+                    help="skip the report of the indexer with factorised query encoders")
     ap.add_argument("--shard", action="store_true",
                     help="under torchrun: split the batch's sequences over the ranks "
                          "(strong scaling of one workload) instead of one replica per GPU")
@@ -277,6 +279,57 @@ def index_launch_ms(dec, inp, reps=20, rounds=5):
     torch.cuda.synchronize()
     del g
     return a.elapsed_time(b) / (reps * rounds)
+
+
+def lowrank_index_report(dev, hbm, reps=20, rounds=5):
+    """The indexer with factorised query encoders (q = W_2 (W_1 h), r = 2048) on the
+    1M-token context: device time per launch (back to back in one CUDA graph) and the
+    fraction of the HBM bandwidth for the bytes it must read (W_1, W_2, h, the candidate
+    keys) and write (the ids)."""
+    import torch
+    import lookahead_sparse_kv_lsa_b200 as lsa
+    import lsa_inputs as LI
+    wl = LI.Workload(LI.one_million_lowrank(), with_pool=False)
+    c = wl.cfg
+    nc = max(0, (int(wl.ctx0[0]) - c.W) // c.block)
+    h, w1, w2 = wl.h(0).to(dev), wl.w_1.to(dev), wl.w_2.to(dev)
+    bias = torch.from_numpy(wl.bias).to(dev)
+    k_idx = wl.k_idx.to(dev)
+    off = torch.from_numpy(wl.blk_off[:1]).to(dev)
+    n_cand = torch.tensor([nc], dtype=torch.int32, device=dev)
+    ids = torch.empty((1, nc), dtype=torch.int32, device=dev)
+    cnt = torch.empty(1, dtype=torch.int32, device=dev)
+    ws = torch.zeros(lsa.index_lowrank_workspace_size(1, c.L, c.d_i, c.rank, nc),
+                     dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    call = lambda: lsa.lsa_index_lowrank(h, w1, w2, bias, k_idx, off, n_cand, nc, ids, cnt, ws, err)
+    call()
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        for _ in range(reps):
+            call()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(rounds):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (reps * rounds)
+    if int(err.item()) != 0:
+        raise SystemExit("device error word %d in the low-rank indexer report" % int(err.item()))
+    n_sel = int(cnt.item())
+    nbytes = (c.L * c.rank * c.D * 2 + c.L * c.d_i * c.rank * 2 + c.L * c.D * 2
+              + nc * c.d_i * 2 + 4 * n_sel)
+    del g
+    return {"workload": "1m_b20_lr2048: B=1, 1M tokens, q = W_2 (W_1 h), W_1 [3][2048][4096], "
+                        "W_2 [3][128][2048], bias -2",
+            "ms": ms, "timing": "%d launches back to back in one graph" % reps,
+            "algorithmic_bytes": nbytes, "achieved_GBs": nbytes / (ms * 1e-3) / 1e9,
+            "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "kept_blocks": n_sel}
 
 
 def index_bytes(cfg, n_cand, n_sel):
@@ -803,6 +856,8 @@ def run_lsa(args, rank, world, local):
         # the oracle leg also checks the timed run's last step and selection
         line["parity_spot_check_max_abs"] = spot_check(wl, out, dec)
         line["near_ties"]["oracle"] = oracle_flips(wl, dec)
+    if rank == 0 and world == 1 and cfg.name == DEFAULT_WORKLOAD and not args.no_lowrank:
+        line["indexer_lowrank"] = lowrank_index_report(dev, hbm)
     if cfg.passes > 1:
         line["delta_gather"] = delta_gather_report(wl, dev)
     if rank == 0 and world == 1 and not args.no_denoise:

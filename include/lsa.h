@@ -122,6 +122,32 @@ lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const float* bia
                         float* logits, uint32_t* layer_mask,
                         void* ws, size_t ws_bytes, int32_t* err, void* stream);
 
+/* lsa_index_lowrank -- lsa_index_ex with factorised query encoders (section 4 of
+ * "FlashMemory-DeepSeek-V4 Explained": a "low-rank query projection (r=2048)"; read here
+ * as each layer's encoder being two stacked linear maps through an r-wide latent):
+ *
+ *   u_l = W_1[l] . h[l][b]          (fp32 accumulation, kept in fp32)
+ *   q_l = W_2[l] . u_l              (fp32 accumulation)
+ *
+ * then scoring, sign test, OR and compaction exactly as lsa_index_ex.
+ *   w_1   device bf16 [L][r][D]     down-projection
+ *   w_2   device bf16 [L][d_i][r]   up-projection
+ *   ws    device workspace of lsa_index_lowrank_workspace_size(B, L, d_i, r, max_cand)
+ *         bytes (16-byte aligned, zero-filled before the first call; the same barrier
+ *         counter rule as lsa_index, three grid barriers per call)
+ * Supported: as lsa_index_ex, plus 256 <= r <= 8192, r % 256 == 0, D <= 16384. The W_1
+ * stream (L r D 2 bytes) dominates the bytes read.
+ */
+lsa_status lsa_index_lowrank(const uint16_t* h, const uint16_t* w_1, const uint16_t* w_2,
+                             int32_t r, const float* bias, const uint16_t* k_idx,
+                             int64_t kidx_layer_stride, const int64_t* kidx_off,
+                             const int32_t* n_cand, int32_t B, int32_t L, int32_t D,
+                             int32_t d_i, int32_t max_cand, int32_t* sel_ids, int32_t* sel_cnt,
+                             int32_t cap, float* logits, uint32_t* layer_mask,
+                             void* ws, size_t ws_bytes, int32_t* err, void* stream);
+size_t lsa_index_lowrank_workspace_size(int32_t B, int32_t L, int32_t d_i, int32_t r,
+                                        int32_t max_cand);
+
 /* ---------------------------------------------------------------------------------
  * lsa_gather -- move the kept blocks from the host cold pool into the HBM pool
  * (section 2 step 3) and build each sequence's block table.

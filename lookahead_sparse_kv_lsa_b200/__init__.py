@@ -14,7 +14,7 @@ import torch
 from . import _lib
 from ._lib import LsaError, LsaState, BLOCK, TAU
 
-__all__ = ["lsa_index", "lsa_gather", "lsa_gather_delta", "lsa_decode_attn", "lsa_step",
+__all__ = ["lsa_index", "lsa_index_lowrank", "index_lowrank_workspace_size", "lsa_gather", "lsa_gather_delta", "lsa_decode_attn", "lsa_step",
            "lsa_load_window", "gather_delta_workspace_size", "lsa_denoise_labels",
            "DENOISE_MAX_BLOCKS", "lsa_wait_selftest",
            "lsa_pass_setup", "lsa_append", "lsa_decode_step",
@@ -84,6 +84,32 @@ def lsa_index(h, w_q, bias, k_idx, kidx_off, n_cand, max_cand: int, sel_ids, sel
         _opt(layer_mask, torch.int32, "layer_mask", (L + 1) * B * ((max_cand + 31) // 32)),
         _dev(ws, torch.uint8, "ws"), ws.numel(), _dev(err, torch.int32, "err", 1), _stream(stream))
     _lib.check("lsa_index", st)
+
+
+def index_lowrank_workspace_size(B: int, L: int, d_i: int, r: int, max_cand: int) -> int:
+    return int(_lib.lib().lsa_index_lowrank_workspace_size(B, L, d_i, r, max_cand))
+
+
+def lsa_index_lowrank(h, w_1, w_2, bias, k_idx, kidx_off, n_cand, max_cand: int, sel_ids,
+                      sel_cnt, ws, err, logits=None, layer_mask=None, stream=None) -> None:
+    """One indexer pass with factorised query encoders q = W_2 (W_1 h); see
+    lsa_index_lowrank in include/lsa.h. w_1 [L][r][D], w_2 [L][d_i][r]."""
+    L, B, D = h.shape
+    r = w_1.shape[1]
+    d_i = w_2.shape[1]
+    cap = sel_ids.shape[1] if sel_ids.dim() == 2 else 0
+    layer_stride = k_idx.shape[1] if k_idx.dim() == 3 else 0
+    st = _lib.lib().lsa_index_lowrank(
+        _dev(h, torch.bfloat16, "h"), _dev(w_1, torch.bfloat16, "w_1", L * r * D),
+        _dev(w_2, torch.bfloat16, "w_2", L * d_i * r), r,
+        _dev(bias, torch.float32, "bias", B), _dev(k_idx, torch.bfloat16, "k_idx"), layer_stride,
+        _dev(kidx_off, torch.int64, "kidx_off", B), _dev(n_cand, torch.int32, "n_cand", B),
+        B, L, D, d_i, max_cand,
+        _dev(sel_ids, torch.int32, "sel_ids"), _dev(sel_cnt, torch.int32, "sel_cnt", B), cap,
+        _opt(logits, torch.float32, "logits", L * B * max_cand),
+        _opt(layer_mask, torch.int32, "layer_mask", (L + 1) * B * ((max_cand + 31) // 32)),
+        _dev(ws, torch.uint8, "ws"), ws.numel(), _dev(err, torch.int32, "err", 1), _stream(stream))
+    _lib.check("lsa_index_lowrank", st)
 
 
 def lsa_gather(host_pool, host_blk_off, sel_ids, sel_cnt, res_pages, n_res, hbm_pool,

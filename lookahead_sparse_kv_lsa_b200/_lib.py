@@ -59,6 +59,9 @@ SIGNATURES = {
     "lsa_index_ex": (_i32, [_p, _p, _p, _p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p,
                             _i32, _p, _p, _p, _sz, _p, _p]),
     "lsa_index_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
+    "lsa_index_lowrank": (_i32, [_p, _p, _p, _i32, _p, _p, _i64, _p, _p, _i32, _i32, _i32, _i32,
+                                 _i32, _p, _p, _i32, _p, _p, _p, _sz, _p, _p]),
+    "lsa_index_lowrank_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "lsa_gather": (_i32, [_p, _i64, _p, _p, _p, _i32, _p, _p, _i32, _i32, _i32, _p, _i64, _i32,
                           _i32, _p, _i32, _p, _p, _p]),
     "lsa_gather_delta": (_i32, [_p, _i64, _p, _p, _p, _i32, _p, _p, _i32, _i32, _i32, _p, _i64,

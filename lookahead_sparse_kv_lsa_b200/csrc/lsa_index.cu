@@ -50,7 +50,10 @@ constexpr int KW = 4;                               // warps that copy K_idx row
 
 struct Args {
   const uint16_t* h;         // [L][B][D]
-  const uint16_t* w_q;       // [L][D_I][D]
+  const uint16_t* w_q;       // [L][D_I][D]; with the factorised encoder W_2 [L][D_I][r]
+  const uint16_t* w_1;       // nullable: factorised encoder, W_1 [L][r][D]
+  float* u;                  // workspace [L][B][r]: the latent W_1 h (factorised encoder)
+  int r;                     // latent width of the factorised encoder (0: none)
   const float* bias;         // [B]
   const uint16_t* k_idx;     // [rows][D_I]; table t of per-layer keys at row t * kls
   long long kls;             // rows between the per-layer key tables (0: one shared table)
@@ -59,7 +62,8 @@ struct Args {
   const int32_t* n_cand;     // [B]
   float* q;                  // workspace [L][B][D_I]
   uint32_t* words;           // workspace [B][n_words]: OR keep bits
-  unsigned long long* sync;  // workspace: grid-barrier arrivals (grows by 2 x grid per launch)
+  unsigned long long* sync;  // workspace: grid-barrier arrivals (grows by one grid size
+                             // per barrier: 2 per launch, 3 with the factorised encoder)
   int32_t* sel_ids;          // [B][cap]
   int32_t* sel_cnt;          // [B]
   float* logits;             // nullable [L][B][max_cand]
@@ -96,6 +100,8 @@ struct Smem {
 };
 
 static_assert(sizeof(Smem) + 128 <= 227 * 1024, "shared memory per CTA");
+// the factorised encoder stages hidden states of up to 16,384 elements in the query buffer
+static_assert(sizeof(float) * CHUNK_WORDS * MAX_L * D_I >= 16384 * 2, "hidden-state staging");
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -357,12 +363,30 @@ __device__ __forceinline__ uint32_t score_word_any(const Args& a, Smem* s, int k
 // Warps KW.. (PROJ_THREADS threads, named barrier 1): q rows [r_lo, r_hi) of the stacked
 // W_q (row = l * D_I + j) for every sequence. Each dot product is cut into NPART parts of
 // whole 8-element groups; a warp sums one part (lane-strided, then a butterfly), and the
-// parts are added in order.
+// parts are added in order. The input vector is h (bf16, D wide) or, for the factorised
+// encoder's second stage, the fp32 latent u (r wide, written earlier in this launch, so
+// it is read through L2).
 constexpr int PROJ_THREADS = NTHREADS - 32 * KW;
 constexpr int PROJ_WARPS = PROJ_THREADS / 32;
+
+template <bool F32_IN>
+__device__ __forceinline__ void load8(const Args& a, int l, int b, int n, int g, float (&f)[8]) {
+  if constexpr (F32_IN) {
+    const float4* v = reinterpret_cast<const float4*>(a.u + (static_cast<long long>(l) * a.B + b) * n) + 2 * g;
+    const float4 x = __ldcg(v), y = __ldcg(v + 1);
+    f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+    f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
+  } else {
+    const uint4* v = reinterpret_cast<const uint4*>(a.h + (static_cast<long long>(l) * a.B + b) * n);
+    unpack8(__ldg(v + g), f);
+  }
+}
+
+template <bool F32_IN>
 __device__ __forceinline__ void project_rows(const Args& a, Smem* s, int r_lo, int r_hi) {
   const int tid = threadIdx.x - 32 * KW, warp = tid >> 5, lane = tid & 31;
-  const int g8 = a.D / 8;
+  const int n = F32_IN ? a.r : a.D;
+  const int g8 = n / 8;
   for (int rg = r_lo; rg < r_hi; rg += RMAX) {
     const int nr = min(RMAX, r_hi - rg);
     for (int b0 = 0; b0 < a.B; b0 += BCH) {
@@ -374,16 +398,14 @@ __device__ __forceinline__ void project_rows(const Args& a, Smem* s, int r_lo, i
         const int bl = rb % nb, r = rb / nb;
         const int row = rg + r;
         const int l = row / D_I;
-        const uint4* wrow = reinterpret_cast<const uint4*>(a.w_q + static_cast<long long>(row) * a.D);
-        const uint4* hrow =
-            reinterpret_cast<const uint4*>(a.h + (static_cast<long long>(l) * a.B + b0 + bl) * a.D);
+        const uint4* wrow = reinterpret_cast<const uint4*>(a.w_q + static_cast<long long>(row) * n);
         const int g_lo = (p * g8) / NPART, g_hi = ((p + 1) * g8) / NPART;
         float acc = 0.f;
 #pragma unroll 4
         for (int g = g_lo + lane; g < g_hi; g += 32) {
           float wf[8], hf[8];
           unpack8(__ldg(wrow + g), wf);
-          unpack8(__ldg(hrow + g), hf);
+          load8<F32_IN>(a, l, b0 + bl, n, g, hf);
 #pragma unroll
           for (int e = 0; e < 8; ++e) acc = fmaf(wf[e], hf[e], acc);
         }
@@ -403,6 +425,76 @@ __device__ __forceinline__ void project_rows(const Args& a, Smem* s, int r_lo, i
       }
       named_bar_sync(1, PROJ_THREADS);
     }
+  }
+}
+
+// First stage of the factorised encoder, all NTHREADS threads: u[l][b][k] = W_1[l][k] .
+// h[l][b] in fp32 for the rows [k_lo, k_hi) of the stacked W_1 (row = l * r + k), one warp
+// per row at a time. The hidden states of a layer are staged in shared memory a group of
+// up to LR_SEQ sequences at a time (the query buffer is idle in this phase); each lane
+// keeps its slice of the W_1 row in registers while it serves the whole group, and a
+// row's dot product is the lanes' fixed-order partial sums joined by a butterfly.
+constexpr int LR_BATCH = 16;                        // 16-byte W_1 pieces per lane in flight
+constexpr int LR_SEQ = 4;                           // sequences per staged group
+__device__ __forceinline__ void lowrank_rows(const Args& a, Smem* s, int k_lo, int k_hi) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint4* hs = reinterpret_cast<uint4*>(&s->qs[0][0][0]);
+  constexpr int HS_CAP = static_cast<int>(sizeof(s->qs) / sizeof(uint4));   // 16-byte slots
+  const int g8 = a.D / 8;                           // 16-byte pieces per row (<= HS_CAP)
+  const int gsz = max(1, min(LR_SEQ, HS_CAP / g8)); // sequences staged at once
+  int row = k_lo;
+  while (row < k_hi) {
+    const int l = row / a.r;
+    const int seg_hi = min(k_hi, (l + 1) * a.r);   // this range's rows of layer l
+    for (int b0 = 0; b0 < a.B; b0 += gsz) {
+      const int nb = min(gsz, a.B - b0);
+      __syncthreads();                              // the previous group's readers are done
+      const uint4* src = reinterpret_cast<const uint4*>(a.h + (static_cast<long long>(l) * a.B + b0) * a.D);
+      for (int i = threadIdx.x; i < nb * g8; i += NTHREADS) hs[i] = __ldg(src + i);
+      __syncthreads();
+      for (int k = row + warp; k < seg_hi; k += NWARPS) {
+        const uint4* wrow = reinterpret_cast<const uint4*>(a.w_1 + static_cast<long long>(k) * a.D);
+        float acc[LR_SEQ];
+#pragma unroll
+        for (int e = 0; e < LR_SEQ; ++e) acc[e] = 0.f;
+        for (int g0 = 0; g0 < g8; g0 += 32 * LR_BATCH) {
+          uint4 w[LR_BATCH];
+#pragma unroll
+          for (int t = 0; t < LR_BATCH; ++t) {
+            const int g = g0 + lane + 32 * t;
+            w[t] = g < g8 ? __ldg(wrow + g) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int t = 0; t < LR_BATCH; ++t) {
+            const int g = g0 + lane + 32 * t;
+            if (g < g8) {
+              float wf[8];
+              unpack8(w[t], wf);
+#pragma unroll
+              for (int e = 0; e < LR_SEQ; ++e) {
+                if (e < nb) {
+                  float hf[8];
+                  unpack8(hs[e * g8 + g], hf);
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) acc[e] = fmaf(wf[i], hf[i], acc[e]);
+                }
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < LR_SEQ; ++e) {
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int e = 0; e < LR_SEQ; ++e)
+            if (e < nb) a.u[(static_cast<long long>(l) * a.B + b0 + e) * a.r + (k - l * a.r)] = acc[e];
+        }
+      }
+    }
+    row = seg_hi;
   }
 }
 
@@ -484,9 +576,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
     const long long NW = s->nw_total;
     const long long W0 = (cta * NW) / G, W1 = ((cta + 1) * NW) / G;
     if (W1 > W0) copy_chunk(a, s, W0, W1 < W0 + ccap ? W1 : W0 + ccap, tid);
-  } else {
+  } else if (a.w_1 == nullptr) {
     const int RQ = a.L * D_I;
-    project_rows(a, s, static_cast<int>((cta * RQ) / G), static_cast<int>(((cta + 1) * RQ) / G));
+    project_rows<false>(a, s, static_cast<int>((cta * RQ) / G), static_cast<int>(((cta + 1) * RQ) / G));
+  }
+  if (a.w_1 != nullptr) {
+    // factorised encoder: the latent u = W_1 h by all warps (the copy warps join once
+    // their K_idx copies are issued), a grid barrier, then q = W_2 u
+    const long long RU = static_cast<long long>(a.L) * a.r;
+    lowrank_rows(a, s, static_cast<int>((cta * RU) / G), static_cast<int>(((cta + 1) * RU) / G));
+    grid_sync(a, s);
+    if (warp >= KW && !s->abort) {
+      const int RQ = a.L * D_I;
+      project_rows<true>(a, s, static_cast<int>((cta * RQ) / G), static_cast<int>(((cta + 1) * RQ) / G));
+    }
   }
   grid_sync(a, s);
   const long long NW = s->nw_total;
@@ -567,21 +670,23 @@ namespace {
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace: the 64-bit grid-barrier counter on its own 256-byte line at the start (zero
-// before the first call; each call adds 2 x grid), then q fp32 [L][B][d_i] and the keep
-// words u32 [B][n_words]. The counter's place does not depend on the shape.
+// before the first call; each call adds one grid size per barrier), then q fp32
+// [L][B][d_i], the keep words u32 [B][n_words] and, for the factorised encoder, the latent
+// u fp32 [L][B][r]. The counter's place does not depend on the shape.
 struct IndexWsLayout {
-  size_t q_off, words_off, sync_off, total;
+  size_t q_off, words_off, u_off, sync_off, total;
   int n_words;
 };
 
-IndexWsLayout index_ws_layout(int B, int L, int max_cand) {
+IndexWsLayout index_ws_layout(int B, int L, int max_cand, int r) {
   IndexWsLayout s;
   s.n_words = (max_cand + 31) / 32;
   if (s.n_words < 1) s.n_words = 1;
   s.sync_off = 0;
   s.q_off = 256;
   s.words_off = align256(s.q_off + static_cast<size_t>(L) * B * lsa::idx::D_I * sizeof(float));
-  s.total = align256(s.words_off + static_cast<size_t>(B) * s.n_words * sizeof(uint32_t));
+  s.u_off = align256(s.words_off + static_cast<size_t>(B) * s.n_words * sizeof(uint32_t));
+  s.total = align256(s.u_off + static_cast<size_t>(L) * B * (r > 0 ? r : 0) * sizeof(float));
   return s;
 }
 
@@ -590,17 +695,18 @@ constexpr size_t kIndexSmem = sizeof(lsa::idx::Smem) + 128;   // + alignment sla
 
 extern "C" size_t lsa_index_workspace_size(int32_t B, int32_t L, int32_t d_i, int32_t max_cand) {
   if (B <= 0 || L <= 0 || d_i != lsa::idx::D_I || max_cand < 0) return 0;
-  return index_ws_layout(B, L, max_cand).total;
+  return index_ws_layout(B, L, max_cand, 0).total;
 }
 
-extern "C" lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const float* bias,
-                                   const uint16_t* k_idx, int64_t kidx_layer_stride,
-                                   const int64_t* kidx_off, const int32_t* n_cand, int32_t B,
-                                   int32_t L, int32_t D, int32_t d_i, int32_t max_cand,
-                                   int32_t* sel_ids, int32_t* sel_cnt, int32_t cap, float* logits,
-                                   uint32_t* layer_mask, void* ws, size_t ws_bytes, int32_t* err,
-                                   void* stream) {
-  lsa_host::NvtxRange nvtx_range("lsa_index");
+namespace {
+// One indexer launch. w_1 == nullptr: the query encoders are w_q [L][d_i][D]; otherwise
+// they are factorised, w_1 [L][r][D] then w_q = W_2 [L][d_i][r].
+lsa_status index_launch(const uint16_t* h, const uint16_t* w_q, const uint16_t* w_1, int32_t r,
+                        const float* bias, const uint16_t* k_idx, int64_t kidx_layer_stride,
+                        const int64_t* kidx_off, const int32_t* n_cand, int32_t B, int32_t L,
+                        int32_t D, int32_t d_i, int32_t max_cand, int32_t* sel_ids,
+                        int32_t* sel_cnt, int32_t cap, float* logits, uint32_t* layer_mask,
+                        void* ws, size_t ws_bytes, int32_t* err, void* stream) {
   if (!h || !w_q || !bias || !k_idx || !kidx_off || !n_cand || !sel_cnt || !ws || !err)
     return LSA_ERR_INVALID_ARG;
   if (kidx_layer_stride < 0) return LSA_ERR_INVALID_ARG;
@@ -611,7 +717,10 @@ extern "C" lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const
   if ((reinterpret_cast<uintptr_t>(h) | reinterpret_cast<uintptr_t>(w_q) |
        reinterpret_cast<uintptr_t>(k_idx) | reinterpret_cast<uintptr_t>(ws)) & 15u)
     return LSA_ERR_INVALID_ARG;
-  const IndexWsLayout lay = index_ws_layout(B, L, max_cand);
+  if (w_1 != nullptr && (r < 256 || r > 8192 || r % 256 != 0 || D > 16384 ||
+                        (reinterpret_cast<uintptr_t>(w_1) & 15u)))
+    return LSA_ERR_INVALID_ARG;
+  const IndexWsLayout lay = index_ws_layout(B, L, max_cand, w_1 != nullptr ? r : 0);
   if (ws_bytes < lay.total) return LSA_ERR_INVALID_ARG;
   const int n_sm = lsa_host::sm_count();
   if (n_sm <= 0) return LSA_ERR_CUDA;
@@ -626,6 +735,9 @@ extern "C" lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const
   lsa::idx::Args a;
   a.h = h;
   a.w_q = w_q;
+  a.w_1 = w_1;
+  a.r = w_1 != nullptr ? r : 0;
+  a.u = w_1 != nullptr ? reinterpret_cast<float*>(base + lay.u_off) : nullptr;
   a.bias = bias;
   a.k_idx = k_idx;
   a.kls = kidx_layer_stride;
@@ -666,6 +778,42 @@ extern "C" lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const
     return LSA_ERR_CUDA;
   }
   return LSA_OK;
+}
+
+}  // namespace
+
+extern "C" lsa_status lsa_index_ex(const uint16_t* h, const uint16_t* w_q, const float* bias,
+                                   const uint16_t* k_idx, int64_t kidx_layer_stride,
+                                   const int64_t* kidx_off, const int32_t* n_cand, int32_t B,
+                                   int32_t L, int32_t D, int32_t d_i, int32_t max_cand,
+                                   int32_t* sel_ids, int32_t* sel_cnt, int32_t cap, float* logits,
+                                   uint32_t* layer_mask, void* ws, size_t ws_bytes, int32_t* err,
+                                   void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_index");
+  return index_launch(h, w_q, nullptr, 0, bias, k_idx, kidx_layer_stride, kidx_off, n_cand, B, L,
+                      D, d_i, max_cand, sel_ids, sel_cnt, cap, logits, layer_mask, ws, ws_bytes,
+                      err, stream);
+}
+
+extern "C" size_t lsa_index_lowrank_workspace_size(int32_t B, int32_t L, int32_t d_i, int32_t r,
+                                                   int32_t max_cand) {
+  if (B <= 0 || L <= 0 || d_i != lsa::idx::D_I || r <= 0 || max_cand < 0) return 0;
+  return index_ws_layout(B, L, max_cand, r).total;
+}
+
+extern "C" lsa_status lsa_index_lowrank(const uint16_t* h, const uint16_t* w_1,
+                                        const uint16_t* w_2, int32_t r, const float* bias,
+                                        const uint16_t* k_idx, int64_t kidx_layer_stride,
+                                        const int64_t* kidx_off, const int32_t* n_cand,
+                                        int32_t B, int32_t L, int32_t D, int32_t d_i,
+                                        int32_t max_cand, int32_t* sel_ids, int32_t* sel_cnt,
+                                        int32_t cap, float* logits, uint32_t* layer_mask,
+                                        void* ws, size_t ws_bytes, int32_t* err, void* stream) {
+  lsa_host::NvtxRange nvtx_range("lsa_index_lowrank");
+  if (!w_1 || !w_2) return LSA_ERR_INVALID_ARG;
+  return index_launch(h, w_2, w_1, r, bias, k_idx, kidx_layer_stride, kidx_off, n_cand, B, L, D,
+                      d_i, max_cand, sel_ids, sel_cnt, cap, logits, layer_mask, ws, ws_bytes, err,
+                      stream);
 }
 
 extern "C" lsa_status lsa_index(const uint16_t* h, const uint16_t* w_q, const float* bias,

@@ -34,6 +34,8 @@ class LsaConfig:
     bias: Optional[List[float]] = None       # per-sequence indexer bias (shared by layers)
     bias_uniform: Optional[tuple] = None     # (lo, hi), drawn per sequence
     kidx_per_layer: bool = False             # one compressed key table per indexer layer
+    rank: int = 0                            # > 0: factorised query encoders W_2 (W_1 h)
+                                             #   through a rank-`rank` latent
     L: int = N_LAYERS
     d_i: int = D_INDEX
     block: int = BLOCK
@@ -93,6 +95,14 @@ def one_million_latent() -> LsaConfig:
     return _fixed("1m_b20_r2048", 1, 1 << 20, 2048, 8192, 64, 512, -2.0, 1, 0)
 
 
+def one_million_lowrank() -> LsaConfig:
+    """1M-token sequence at bias -2 whose query encoders are factorised through a rank-2048
+    latent: q = W_2 (W_1 h), W_1 [3][2048][4096], W_2 [3][128][2048]."""
+    c = _fixed("1m_b20_lr2048", 1, 1 << 20, 4096, 8192, 64, 512, -2.0, 1, 0)
+    c.rank = 2048
+    return c
+
+
 def ragged_mix() -> LsaConfig:
     """B=64, context U{512..4096} blocks per sequence, bias U(-3,-1) per sequence, seed 7."""
     return LsaConfig(name="ragged_b64", B=64, D=4096, W=4096, H=64, d=512, passes=1, seed=7,
@@ -101,7 +111,8 @@ def ragged_mix() -> LsaConfig:
 
 def all_configs() -> List[LsaConfig]:
     return [tiny(), mid_batch(), long_ctx(), one_million(-1.5), one_million(-2.0),
-            one_million(-2.5), ragged_mix(), one_million_layer_keys(), one_million_latent()]
+            one_million(-2.5), ragged_mix(), one_million_layer_keys(), one_million_latent(),
+            one_million_lowrank()]
 
 
 def by_name(name: str) -> LsaConfig:

@@ -93,6 +93,13 @@ class Workload:
         self.total_blocks = int(off[-1])
 
         self.w_q = _randn_bf16((cfg.L, cfg.d_i, cfg.D), _gen(cfg.seed, "w_q"), cfg.wq_std)
+        self.w_1 = self.w_2 = None
+        if cfg.rank > 0:
+            # factorised encoders: W_1 ~ N(0, 1/D), W_2 ~ N(0, 1/rank) (variance-preserving)
+            self.w_1 = _randn_bf16((cfg.L, cfg.rank, cfg.D), _gen(cfg.seed, "w_1"),
+                                   cfg.D ** -0.5)
+            self.w_2 = _randn_bf16((cfg.L, cfg.d_i, cfg.rank), _gen(cfg.seed, "w_2"),
+                                   cfg.rank ** -0.5)
         gb = [int(x) for x in self.seqs]          # global sequence index of each row
         if cfg.kidx_per_layer:
             # one table per layer: [L][blocks][d_i]

@@ -77,6 +77,19 @@ def query_projection(w_q: np.ndarray, h: np.ndarray) -> np.ndarray:
     return np.stack([w_q[l] @ h[l] for l in range(L)])
 
 
+def query_projection_lowrank(w_1: np.ndarray, w_2: np.ndarray, h: np.ndarray) -> np.ndarray:
+    """q_l = W_2,l . (W_1,l . h_l): each layer's query encoder factorised through a rank-r
+    latent (the "low-rank query projection (r=2048)" of section 4 of the zhichai.net
+    explainer, read as two stacked linear maps).
+
+    w_1: [L][r][D] (down-projection), w_2: [L][d_i][r] (up-projection), h: [L][D].
+    returns q: [L][d_i]. The latent W_1,l . h_l is kept exact (float64), not rounded.
+    """
+    L = w_1.shape[0]
+    assert w_2.shape[0] == L and w_2.shape[2] == w_1.shape[1] and h.shape == (L, w_1.shape[2])
+    return np.stack([w_2[l] @ (w_1[l] @ h[l]) for l in range(L)])
+
+
 def block_logits(q: np.ndarray, k_idx: np.ndarray, bias: float) -> np.ndarray:
     """z_l[c] = q_l . K_idx[c] / sqrt(d_i) + bias, for every layer l and block c.
 
@@ -112,6 +125,15 @@ def index_pass(w_q_bits, h_bits, k_idx_bits, bias: float):
     (ids, z) with z float64 [L][n_cand].
     """
     q = query_projection(bf16_to_f64(w_q_bits), bf16_to_f64(h_bits))
+    z = block_logits(q, bf16_to_f64(k_idx_bits), float(bias))
+    return kept_blocks(z), z
+
+
+def index_pass_lowrank(w_1_bits, w_2_bits, h_bits, k_idx_bits, bias: float):
+    """index_pass with the factorised query encoder: w_1_bits [L][r][D], w_2_bits
+    [L][d_i][r] (bf16 bit patterns); the rest as index_pass. Returns (ids, z)."""
+    q = query_projection_lowrank(bf16_to_f64(w_1_bits), bf16_to_f64(w_2_bits),
+                                 bf16_to_f64(h_bits))
     z = block_logits(q, bf16_to_f64(k_idx_bits), float(bias))
     return kept_blocks(z), z
 

@@ -152,3 +152,66 @@ def test_many_short_sequences(cuda_ok):
         # the barrier counter (first 8 bytes) grew by two rounds of the grid per call
         assert int(ws[:8].cpu().view(torch.int64)[0]) == 2 * G * (call + 1)
         assert not ws[8:256].any()
+
+
+def run_index_lowrank(wl, p, calls=1):
+    """lsa_index_lowrank on pass p of a workload with factorised encoders; returns the
+    last call's (ids, counts, logits, err, n_cand, workspace)."""
+    dev = torch.device("cuda")
+    c = wl.cfg
+    B, L = c.B, c.L
+    n_cand = [oracle.n_candidates(int(x), c.W) for x in wl.ctx_at(p)]
+    max_cand = max(1, max(n_cand))
+    sel_ids = torch.full((B, max_cand), -1, dtype=torch.int32, device=dev)
+    sel_cnt = torch.full((B,), -1, dtype=torch.int32, device=dev)
+    logits = torch.full((L, B, max_cand), float("nan"), device=dev)
+    ws = torch.zeros(lsa.index_lowrank_workspace_size(B, L, c.d_i, c.rank, max_cand),
+                     dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    args = (wl.h(p).to(dev), wl.w_1.to(dev), wl.w_2.to(dev), torch.from_numpy(wl.bias).to(dev),
+            wl.k_idx.to(dev), torch.from_numpy(wl.blk_off[:B]).to(dev),
+            torch.tensor(n_cand, dtype=torch.int32, device=dev), max_cand, sel_ids, sel_cnt, ws, err)
+    for _ in range(calls):
+        lsa.lsa_index_lowrank(*args, logits=logits)
+    torch.cuda.synchronize()
+    return sel_ids.cpu(), sel_cnt.cpu(), logits.cpu().numpy(), int(err.item()), n_cand, ws
+
+
+def check_lowrank(wl, calls=1):
+    c = wl.cfg
+    ids, cnt, z_gpu, err, n_cand, ws = run_index_lowrank(wl, 0, calls)
+    assert err == 0
+    w1, w2, hb = bits(wl.w_1), bits(wl.w_2), bits(wl.h(0))
+    n_near = 0
+    for b in range(c.B):
+        nc = n_cand[b]
+        ref_ids, z_ref = oracle.index_pass_lowrank(w1, w2, hb[:, b], cand_keys(wl, b, nc),
+                                                   float(wl.bias[b]))
+        dz = np.abs(z_gpu[:, b, :nc] - z_ref)
+        assert dz.max(initial=0.0) <= LOGIT_ABS, (c.name, b, dz.max())
+        got = ids[b, :int(cnt[b])].tolist()
+        n_near += len(compare_selection(got, ref_ids, z_ref, "%s b%d" % (c.name, b)))
+        assert got == np.flatnonzero((z_gpu[:, b, :nc] > 0).any(axis=0)).tolist()
+    assert n_near <= max(3, 0.01 * sum(n_cand))
+    return ws
+
+
+def test_lowrank_encoder_full_size(cuda_ok):
+    """Factorised query encoders q = W_2 (W_1 h), r = 2048, D = 4096, at the 1M-token
+    context: logits within the tolerance of the oracle's float64 values, ids exact
+    outside the near-tie band."""
+    check_lowrank(LI.Workload(LI.one_million_lowrank(), with_pool=False))
+
+
+def test_lowrank_encoder_batch_and_small_rank(cuda_ok):
+    """Five sequences (more than one staged group of hidden states), D = 1024, r = 512
+    (a CTA's latent rows span two layers), two calls on one workspace: the barrier
+    counter grows by three rounds of the grid per call."""
+    import dataclasses
+    cfg = LI.scaled_down(LI.one_million_lowrank(), ctx_blocks=300, B=5)
+    cfg = dataclasses.replace(cfg, D=1024, rank=512)
+    cfg.bias = [-2.0, -1.0, -3.0, -1.5, -2.5]
+    wl = LI.Workload(cfg, with_pool=False)
+    ws = check_lowrank(wl, calls=2)
+    G = min(torch.cuda.get_device_properties(0).multi_processor_count, 1024)
+    assert int(ws[:8].cpu().view(torch.int64)[0]) == 3 * G * 2

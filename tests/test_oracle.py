@@ -62,6 +62,52 @@ def check_projection_bruteforce(O=O):
             assert q[l, j] == float(exact)
 
 
+def check_lowrank_reduces_to_full_rank(O=O):
+    """With integer factors, W_2 . (W_1 . h) equals (W_2 W_1) . h exactly: the factorised
+    encoder is the full-rank one whose W_q is the product of its factors."""
+    rng = np.random.default_rng(21)
+    L, d_i, r, D = 3, 6, 10, 16
+    w1 = rng.integers(-4, 5, (L, r, D)).astype(np.float64)
+    w2 = rng.integers(-4, 5, (L, d_i, r)).astype(np.float64)
+    h = rng.integers(-8, 9, (L, D)).astype(np.float64) / 4.0
+    wq = np.stack([(w2[l].astype(np.int64) @ w1[l].astype(np.int64)).astype(np.float64)
+                   for l in range(L)])
+    got = O.query_projection_lowrank(w1, w2, h)
+    assert np.array_equal(got, O.query_projection(wq, h))
+    # and against a brute-force triple loop in exact rationals
+    for l in range(L):
+        for j in range(d_i):
+            acc = Fraction(0)
+            for k in range(r):
+                u = sum(Fraction(w1[l, k, i]) * Fraction(h[l, i]) for i in range(D))
+                acc += Fraction(w2[l, j, k]) * u
+            assert got[l, j] == float(acc)
+
+
+def check_lowrank_unit_rows(O=O):
+    """Unit-row factors pick components: W_1 row k = e_{a(k)}, W_2 row j = e_{b(j)} give
+    q_l[j] = h_l[a(b(j))] in every layer, with the layer's own permutations."""
+    rng = np.random.default_rng(22)
+    L, d_i, r, D = 3, 8, 12, 30
+    w1 = np.zeros((L, r, D)); w2 = np.zeros((L, d_i, r))
+    a = [rng.permutation(D)[:r] for _ in range(L)]
+    b = [rng.permutation(r)[:d_i] for _ in range(L)]
+    for l in range(L):
+        w1[l, np.arange(r), a[l]] = 1.0
+        w2[l, np.arange(d_i), b[l]] = 1.0
+    h = rng.standard_normal((L, D))
+    q = O.query_projection_lowrank(w1, w2, h)
+    for l in range(L):
+        assert np.array_equal(q[l], h[l][a[l][b[l]]])
+    # the whole pass: a block whose key is a unit vector e_j scores q_l[j] / sqrt(d_i) + bias
+    k = np.eye(d_i)
+    ids, z = O.index_pass_lowrank(f64_to_bf16_bits(w1), f64_to_bf16_bits(w2),
+                                  f64_to_bf16_bits(np.round(h * 4) / 4), f64_to_bf16_bits(k), 0.0)
+    hq = O.query_projection_lowrank(w1, w2, np.round(h * 4) / 4)
+    assert np.allclose(z, hq / math.sqrt(d_i), rtol=0, atol=1e-15)
+    assert list(ids) == list(np.flatnonzero((hq > 0).any(axis=0)))
+
+
 def check_logits_closed_form(O=O):
     # d_i = 64 -> sqrt(d_i) = 8 exactly; q = (2, 0, ...), K_idx[c] = (c - 3, 0, ...)
     d_i, n = 64, 9
@@ -329,6 +375,7 @@ def check_vote(O=O):
 
 
 PINS = [check_bf16_decode, check_projection_unit_rows, check_projection_bruteforce,
+        check_lowrank_reduces_to_full_rank, check_lowrank_unit_rows,
         check_logits_closed_form, check_per_layer_keys, check_threshold_strict, check_union_bruteforce,
         check_selection_rate, check_single_token, check_two_token_closed_form,
         check_matches_sdpa, check_chunked_attention_matches_whole, check_uniform_when_q_zero, check_attended_set,
@@ -368,6 +415,12 @@ class _Mutant:
             z = me.block_logits(q, me.bf16_to_f64(k_idx_bits), float(bias))
             return me.kept_blocks(z), z
 
+        def index_pass_lowrank(w1_bits, w2_bits, h_bits, k_idx_bits, bias):
+            q = me.query_projection_lowrank(me.bf16_to_f64(w1_bits), me.bf16_to_f64(w2_bits),
+                                            me.bf16_to_f64(h_bits))
+            z = me.block_logits(q, me.bf16_to_f64(k_idx_bits), float(bias))
+            return me.kept_blocks(z), z
+
         def step_output(q_bits, K_bits, V_bits, ids, n_ctx, window, s, scale, heads=None, block=64):
             pos = me.attended_positions(ids, n_ctx, window, s, block)
             q = me.bf16_to_f64(q_bits)
@@ -385,6 +438,7 @@ class _Mutant:
             return out
 
         self.index_pass = repl.get("index_pass", index_pass)
+        self.index_pass_lowrank = repl.get("index_pass_lowrank", index_pass_lowrank)
         self.step_output = repl.get("step_output", step_output)
         self.decode_sequence = repl.get("decode_sequence", decode_sequence)
 
@@ -417,6 +471,13 @@ MUTANTS = {
         q, k if k.ndim == 2 else np.roll(k, 1, axis=0), b)),
     "per_layer_keys_first_table_only": dict(block_logits=lambda q, k, b: O.block_logits(
         q, k if k.ndim == 2 else k[0], b)),
+    "lowrank_skips_up_projection": dict(query_projection_lowrank=lambda w1, w2, h: np.stack(
+        [(w1[l] @ h[l])[:w2.shape[1]] for l in range(w1.shape[0])])),
+    "lowrank_down_projection_of_next_layer": dict(query_projection_lowrank=lambda w1, w2, h: np.stack(
+        [w2[l] @ (w1[(l + 1) % w1.shape[0]] @ h[l]) for l in range(w1.shape[0])])),
+    "lowrank_latent_rounded_to_bf16": dict(query_projection_lowrank=lambda w1, w2, h: np.stack(
+        [w2[l] @ torch.from_numpy(w1[l] @ h[l]).to(torch.bfloat16).double().numpy()
+         for l in range(w1.shape[0])])),
     "threshold_ge": dict(kept_blocks=lambda z: np.flatnonzero((z >= 0).any(axis=0))),
     "and_instead_of_or": dict(kept_blocks=lambda z: np.flatnonzero((z > 0).all(axis=0))),
     "only_first_layer": dict(kept_blocks=lambda z: np.flatnonzero(z[0] > 0)),
