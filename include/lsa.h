@@ -257,7 +257,7 @@ size_t lsa_decode_attn_workspace_size(int32_t B, int32_t H, int32_t d, int32_t n
  * GPU that loads the library holds until the process exits. The call allocates nothing
  * (no cudaMalloc, cudaFree or allocating library routine).
  *  - Limit: lsa_decode_attn_workspace_size(B, H, d, n_sm) must not exceed
- *    LSA_NOALLOC_SCRATCH_BYTES (e.g. B <= 107 at H = 64, d = 512, 148 SMs); larger
+ *    LSA_NOALLOC_SCRATCH_BYTES (e.g. B <= 106 at H = 64, d = 512, 148 SMs); larger
  *    problems return LSA_ERR_CAPACITY before anything is enqueued.
  *  - The first call on a device looks up the array's device address and enqueues, on
  *    the caller's stream and ahead of the kernel, a clear of the array's first 256

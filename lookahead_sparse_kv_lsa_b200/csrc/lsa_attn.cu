@@ -42,7 +42,7 @@ constexpr int NTHREADS = 192;
 constexpr int MAXSEG = 16;                // segments planned per batch
 constexpr float RESCALE_LOG2 = 8.0f;      // raise the running max only by more than 2^8
 constexpr int MAXITEMS = 64;              // sequences a CTA's merge range meets, per round
-constexpr int MAXRUNS = 32;               // (sequence, head, chunk range) runs per merge group
+constexpr int MAXRUNS = 64;               // (sequence, head, chunk range) runs per merge group
 constexpr int SCRATCH_FLOATS = 4 * NTHREADS;  // merge scratch after a group's rows
 constexpr int MAX_GRID = 256;             // CTAs per launch (one per SM)
 
@@ -54,6 +54,7 @@ struct Misc {
   uint64_t full[NST], empty[NST];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, pv_done, q_full, q_free, mma_done;
+  uint64_t merge_bar;               // the merge's bulk copies of partial rows
   uint32_t tmem_base;
   int abort;
   int nseg, more;
@@ -65,9 +66,10 @@ struct Misc {
   // fused merge
   int n_items, total_items;
   long long merge_j0, merge_j1, cur_j;
-  int cur_rec, n_runs, group_floats;
+  int cur_rec, n_runs, group_floats, precut;
+  long long group_bytes;
   int item_b[MAXITEMS], item_h[MAXITEMS], item_clo[MAXITEMS], item_chi[MAXITEMS];
-  int run_b[MAXRUNS], run_h[MAXRUNS], run_d0[MAXRUNS], run_w[MAXRUNS], run_clo[MAXRUNS],
+  int run_b[MAXRUNS], run_h[MAXRUNS], run_c0[MAXRUNS], run_nch[MAXRUNS], run_clo[MAXRUNS],
       run_n[MAXRUNS], run_off[MAXRUNS];
   float run_inv[MAXRUNS];
   long long ustart[MAX_GRID + 1];   // first unit of each CTA: floor(c * U / G)
@@ -77,8 +79,10 @@ struct Args {
   const int32_t* block_table;
   const int32_t* n_entries;
   const int32_t* tail_len;
-  float* part_o;          // [slots][d/128][H][128] fp32: each 128-dim block contiguous
-  float* part_ml;         // [slots][H][2] fp32 (running max in log2 units, denominator)
+  float* part_o;          // [d/128][H][slots][128] fp32: the rows a merge item needs (one
+                          //   128-dim chunk of one head over consecutive slots) are contiguous
+  float* part_ml;         // [H][slots][4] fp32 (running max in log2 units, denominator, two
+                          //   pad words: 16 bytes, so a run's pairs come by one bulk copy)
   unsigned int* sync;     // [2] grid-barrier arrive / depart counters (left at zero)
   uint16_t* out;          // [B][H][d] bf16
   uint16_t* pool;         // the HBM pool (written only by the fused append)
@@ -242,7 +246,7 @@ __device__ __forceinline__ bool cta_empty(long long c, long long U, long long G)
   return (c * U) / G == ((c + 1) * U) / G;
 }
 
-// Merge work items are (sequence, head, 64-dim chunk) triples of every sequence whose
+// Merge work items are (sequence, head, 128-dim chunk) triples of every sequence whose
 // units span more than one CTA (they are merged from partials) or that has no units at
 // all (its output is zero-filled), numbered in sequence order. CTA c owns the
 // contiguous item range [c*T/G, (c+1)*T/G), so a CTA's items mostly share a head.
@@ -253,7 +257,7 @@ __device__ __forceinline__ bool cta_empty(long long c, long long U, long long G)
 __device__ __noinline__ void plan_merge(const Args& a, long long U, int skip, Misc* m, int lane) {
   const long long G = gridDim.x;
   const int cta = blockIdx.x;
-  const int n_chunks = a.d / 64;
+  const int n_chunks = a.d / 128;
   // pass 1: total items T
   long long T = 0;
   {
@@ -358,21 +362,83 @@ __device__ __forceinline__ float block_sum(float v, Misc* m, int tid, int nwarps
   return r;
 }
 
+constexpr int CW = 128;                   // merge chunk: head dimensions per partial row
+
+// One thread: cut the next group of merge runs (one sequence, one head, a range of
+// 128-dim chunks) from the CTA's recorded items, as many as fit `buf_floats` minus the
+// output scratch. A run's region holds its nch chunks of n rows of CW floats, then n
+// (m, l) pairs, then n weights (16-byte multiples, so that every chunk starts on a
+// 16-byte boundary as bulk copies require). Sets n_runs, group_floats, group_bytes (the
+// bytes the group's bulk copies bring) and advances cur_rec / cur_j.
+__device__ __noinline__ void cut_group(const Args& a, Misc* m, int buf_floats) {
+  const int nrec = m->n_items;
+  const int nch_all = a.d / CW;
+  int r = m->cur_rec, nr = 0;
+  long long j = m->cur_j;
+  long long used = 0, bytes = 0;
+  while (r < nrec && nr < MAXRUNS) {
+    const long long ib = m->item_h[r];
+    const long long lo = m->merge_j0 > ib ? m->merge_j0 : ib;
+    const long long hi_all = ib + static_cast<long long>(a.H) * nch_all;
+    const long long hi = m->merge_j1 < hi_all ? m->merge_j1 : hi_all;
+    if (j < lo) j = lo;
+    if (j >= hi) {
+      ++r;
+      j = -1;
+      continue;
+    }
+    const int rel = static_cast<int>(j - ib);   // < H * nch_all: 32-bit division
+    const int h = rel / nch_all;
+    const int c0 = rel - h * nch_all;
+    long long run_end = ib + static_cast<long long>(h + 1) * nch_all;
+    if (run_end > hi) run_end = hi;
+    int nch = static_cast<int>(run_end - j);
+    const int n = m->item_chi[r] - m->item_clo[r] + 1;   // 0: empty sequence
+    const long long tail = 4LL * n + ((n + 3) & ~3LL);   // (m, l, pad, pad) and weights
+    long long need = static_cast<long long>(nch) * n * CW + tail;
+    if (used + need > buf_floats - SCRATCH_FLOATS) {
+      if (nr > 0) break;
+      nch = static_cast<int>((buf_floats - SCRATCH_FLOATS - tail) / (n > 0 ? static_cast<long long>(CW) * n : 1));
+      if (nch < 1) nch = 1;     // n <= MAX_GRID: one chunk (128 KB) always fits
+      need = static_cast<long long>(nch) * n * CW + tail;
+    }
+    m->run_b[nr] = m->item_b[r];
+    m->run_h[nr] = h;
+    m->run_c0[nr] = c0;
+    m->run_nch[nr] = nch;
+    m->run_clo[nr] = m->item_clo[r];
+    m->run_n[nr] = n;
+    m->run_off[nr] = static_cast<int>(used);
+    used += need;
+    bytes += static_cast<long long>(nch) * n * CW * 4 + 16LL * n;
+    j += nch;
+    ++nr;
+  }
+  m->cur_rec = r;
+  m->cur_j = j;
+  m->n_runs = nr;
+  m->group_floats = static_cast<int>(used);
+  m->group_bytes = bytes;
+}
+
 // Fused log-sum-exp merge, run by every thread of every CTA after its segments:
 //   M = max_k m_k,  out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k   (m in log2 units)
 // over the partials k of a split sequence. A grid-wide barrier (one arrival counter,
 // bounded wait) separates the partial writes from the reads. The CTA's items are cut
-// into runs (one sequence, one head, a range of 64-dim chunks); a group of runs that
-// fits the idle shared memory has all its partial rows fetched with 1-D bulk copies
-// (issued by all threads, one round trip) while one warp per run derives the split
-// weights; then every thread reduces a few output dimensions over the partials.
+// into runs (one sequence, one head, a range of 128-dim chunks; the first group is cut
+// before the barrier). In the partial layout the rows of one chunk of one head over
+// consecutive slots are contiguous, so a run needs one 1-D bulk copy per chunk and one
+// for its (m, l) pairs; all the group's copies are issued at once (spread over the
+// threads): one round trip per group. One warp per run derives the split weights from
+// shared memory; then the threads of a warp take consecutive 16-byte
+// columns of one run and walk the same split rows, each slice of the threads a
+// contiguous range of the splits, and the slices meet in scratch.
 __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, int buf_floats,
                                          long long U, bool aborted) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NWARPS = NTHREADS / 32;
   const long long G = gridDim.x;
-  const int nch = a.d / 64;
-  // m->ustart and the round-0 plan were filled by the producer warp after its last loads
+  const long long S = G + a.B;           // partial slots: CTA + sequence
   if (m->total_items == 0) return;     // nothing split or empty: no barrier, all CTAs agree
   // ---- grid barrier: all partials written before any is read
   if (tid == 0) {
@@ -382,14 +448,16 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
     const bool ok = before + 1u >= static_cast<unsigned int>(G) ||
                     spin_until_geq(a.sync, static_cast<unsigned int>(G));
     __threadfence();
-    fence_proxy_async_global();       // the partials are read back by bulk copies
     if (!ok) {
       set_err(a.err, LSA_DEVERR_TIMEOUT);
       m->abort = 1;
     }
   }
   __syncthreads();
+  fence_proxy_async_global();           // the partials are read back by bulk copies
   bool failed = m->abort != 0 || aborted;   // the same value in every thread
+  const bool precut = m->precut != 0;
+  uint32_t group_no = 0;                 // phases of merge_bar completed so far
   for (int round = 0; !failed; ++round) {
     if (round > 0) {
       __syncthreads();
@@ -398,163 +466,129 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
     }
     const int nrec = m->n_items;
     if (nrec == 0) break;
-    if (tid == 0) {
+    bool first = round == 0 && precut;   // the first group was cut before the barrier
+    if (!first && tid == 0) {
       m->cur_rec = 0;
       m->cur_j = -1;
     }
-    __syncthreads();
     while (!failed) {
-      // ---- thread 0 cuts the next group of runs
       if (tid == 0) {
-        int r = m->cur_rec, nr = 0;
-        long long j = m->cur_j;
-        long long used = 0;
-        while (r < nrec && nr < MAXRUNS) {
-          const long long ib = m->item_h[r];
-          const long long lo = m->merge_j0 > ib ? m->merge_j0 : ib;
-          const long long hi_all = ib + static_cast<long long>(a.H) * nch;
-          const long long hi = m->merge_j1 < hi_all ? m->merge_j1 : hi_all;
-          if (j < lo) j = lo;
-          if (j >= hi) {
-            ++r;
-            j = -1;
-            continue;
-          }
-          const int rel = static_cast<int>(j - ib);   // < H * nch: 32-bit division
-          const int h = rel / nch;
-          const int c0 = rel - h * nch;
-          long long run_end = ib + static_cast<long long>(h + 1) * nch;
-          if (run_end > hi) run_end = hi;
-          int nchunks = static_cast<int>(run_end - j);
-          const int n = m->item_chi[r] - m->item_clo[r] + 1;   // 0: empty sequence
-          // rows, then the n weights padded to 4 floats so that every run's rows start
-          // on a 16-byte boundary (bulk copies require it)
-          const int wpad = (n + 3) & ~3;
-          long long need = static_cast<long long>(n) * (nchunks * 64) + wpad;
-          if (used + need > buf_floats - SCRATCH_FLOATS) {
-            if (nr > 0) break;
-            nchunks = static_cast<int>((buf_floats - SCRATCH_FLOATS - wpad) / (n > 0 ? n : 1) / 64);
-            if (nchunks < 1) nchunks = 1;  // buf_floats >= 256 * 64 + 256 by construction
-            need = static_cast<long long>(n) * (nchunks * 64) + wpad;
-          }
-          m->run_b[nr] = m->item_b[r];
-          m->run_h[nr] = h;
-          m->run_d0[nr] = c0 * 64;
-          m->run_w[nr] = nchunks * 64;
-          m->run_clo[nr] = m->item_clo[r];
-          m->run_n[nr] = n;
-          m->run_off[nr] = static_cast<int>(used);
-          used += need;
-          j += nchunks;
-          ++nr;
-        }
-        m->cur_rec = r;
-        m->cur_j = j;
-        m->n_runs = nr;
-        m->group_floats = static_cast<int>(used);
-
+        if (!first) cut_group(a, m, buf_floats);
+        if (m->group_bytes > 0)
+          mbar_arrive_expect_tx(&m->merge_bar, static_cast<uint32_t>(m->group_bytes));
       }
+      first = false;
       __syncthreads();
       const int nr = m->n_runs;
       if (nr == 0) break;
-      // ---- partial rows: 16-byte asynchronous copies from L2, spread over all threads
-      // (columns across threads, splits down the rows): one round trip for the group
-      for (int q = 0; q < nr; ++q) {
-        const int n = m->run_n[q], w4 = m->run_w[q] >> 2;
-        const int rows_per_pass = NTHREADS / w4;           // run_w <= 512: w4 <= 128
-        const int c = tid % w4, r0 = tid / w4;
-        if (r0 < rows_per_pass) {
+      const bool copies = m->group_bytes > 0;
+      // ---- one bulk copy per (run, chunk), spread over the threads
+      {
+        int q = 0, before = 0;
+        for (int p = tid;; p += NTHREADS) {
+          while (q < nr && p >= before + m->run_nch[q]) before += m->run_nch[q++];
+          if (q >= nr) break;
+          const int n = m->run_n[q];
+          if (n == 0) continue;
+          const int i = p - before;
           const long long b = m->run_b[q], h = m->run_h[q];
-          const uint32_t dst0 = smem_u32(buf + m->run_off[q]) + c * 16;
-          const int x = m->run_d0[q] + 4 * c;       // head dimension of this column
-          const float* src0 = a.part_o + ((x >> 7) * a.H + h) * 128 + (x & 127);
-          for (int k = r0; k < n; k += rows_per_pass) {
-            const long long slot = m->run_clo[q] + k + b;
-            cp_async16(dst0 + static_cast<uint32_t>(k) * (w4 * 16),
-                       src0 + slot * a.H * a.d);
-          }
+          const float* src = a.part_o + ((static_cast<long long>(m->run_c0[q] + i) * a.H + h) * S +
+                                         m->run_clo[q] + b) * CW;
+          bulk_load(buf + m->run_off[q] + static_cast<long long>(i) * n * CW, src,
+                    static_cast<uint32_t>(n) * (CW * 4u), &m->merge_bar);
         }
       }
-      cp_async_commit();
-      // ---- split weights: one warp per run; all (m, l) pairs of a run are loaded in
-      // one batch (up to MAX_GRID / 32 per lane) so the weights cost one round trip
-      for (int q = warp; q < nr; q += NWARPS) {
-        const int n = m->run_n[q], b = m->run_b[q], h = m->run_h[q], clo = m->run_clo[q];
-        float* w = buf + m->run_off[q] + static_cast<long long>(n) * m->run_w[q];
-        constexpr int PER_LANE = MAX_GRID / 32;
-        float2 ml[PER_LANE];
-#pragma unroll
-        for (int i = 0; i < PER_LANE; ++i) {
-          const int k = lane + 32 * i;
-          const long long c = clo + k;
-          ml[i] = make_float2(-INFINITY, 0.f);
-          if (k < n && m->ustart[c] != m->ustart[c + 1])
-            ml[i] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (c + b) * a.H + h);
+      // ---- and one bulk copy of each run's (m, l) quadruples
+      for (int q = tid; q < nr; q += NTHREADS) {
+        const int n = m->run_n[q];
+        if (n == 0) continue;
+        const float* src = a.part_ml + (static_cast<long long>(m->run_h[q]) * S + m->run_clo[q] +
+                                        m->run_b[q]) * 4;
+        bulk_load(buf + m->run_off[q] + static_cast<long long>(m->run_nch[q]) * n * CW, src,
+                  static_cast<uint32_t>(n) * 16u, &m->merge_bar);
+      }
+      bool ok = true;
+      if (copies) ok = mbar_wait(&m->merge_bar, group_no & 1, nullptr);
+      if (copies) ++group_no;
+      if (!__syncthreads_and(ok)) {
+        if (tid == 0) {
+          set_err(a.err, LSA_DEVERR_TIMEOUT);
+          m->abort = 1;
         }
+        failed = true;
+        break;
+      }
+      // ---- split weights, one warp per run, from shared memory; an empty CTA's slot (no
+      // units, nothing written) gets weight 0
+      for (int q = warp; q < nr; q += NWARPS) {
+        const int n = m->run_n[q];
+        const float* ml = buf + m->run_off[q] + static_cast<long long>(m->run_nch[q]) * n * CW;
+        float* w = const_cast<float*>(ml) + 4 * n;
+        const long long c0 = m->run_clo[q];
         float mx = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < PER_LANE; ++i) mx = fmaxf(mx, ml[i].x);
+        for (int k = lane; k < n; k += 32)
+          if (m->ustart[c0 + k] != m->ustart[c0 + k + 1]) mx = fmaxf(mx, ml[4 * k]);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float ls = 0.f;
-#pragma unroll
-        for (int i = 0; i < PER_LANE; ++i) {
-          const int k = lane + 32 * i;
-          const float wk = ml[i].x == -INFINITY ? 0.f : exp2f(ml[i].x - mx);
-          ls += wk * ml[i].y;
-          if (k < n) w[k] = wk;
+        for (int k = lane; k < n; k += 32) {
+          const bool live = m->ustart[c0 + k] != m->ustart[c0 + k + 1];
+          const float mk = ml[4 * k];
+          const float wk = (!live || mk == -INFINITY) ? 0.f : exp2f(mk - mx);
+          ls += wk == 0.f ? 0.f : wk * ml[4 * k + 1];
+          w[k] = wk;
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
         if (lane == 0) m->run_inv[q] = ls > 0.f ? 1.f / ls : 0.f;
       }
-      cp_async_wait_all();
       __syncthreads();
-      // ---- outputs: threads take (run, 4-dim column, split slice) triples; each sums
-      // its slice of the splits with float4 shared loads, the slices meet in scratch
+      // ---- outputs: jobs are (run, chunk, 16-byte column); the threads of a slice take
+      // consecutive columns and walk the same rows, slices split the rows in ranges
       int total_c4 = 0;
-      for (int q = 0; q < nr; ++q) total_c4 += m->run_w[q] >> 2;
+      for (int q = 0; q < nr; ++q) total_c4 += (CW / 4) * m->run_nch[q];
       int slices = NTHREADS / (total_c4 > 0 ? total_c4 : 1);
       slices = slices < 1 ? 1 : (slices > 8 ? 8 : slices);
+      const int per_c = NTHREADS / slices;     // columns per pass
+      const int sl = tid / per_c, t = tid - sl * per_c;
       float4* scratch = reinterpret_cast<float4*>(buf + m->group_floats);
-      for (int base = 0; base < total_c4; base += NTHREADS / slices) {
-        const int per = NTHREADS / slices;
-        const int t = tid / slices, sl = tid - t * slices;
+      for (int base = 0; base < total_c4; base += per_c) {
         const int c4 = base + t;
+        const bool act = sl < slices && c4 < total_c4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        int q = 0;
-        if (t < per && c4 < total_c4) {
+        int q = 0, i = 0, col = 0;
+        if (act) {
           int x = c4;
-          while (x >= (m->run_w[q] >> 2)) x -= m->run_w[q++] >> 2;
-          const int n = m->run_n[q], wq = m->run_w[q];
-          const float* rows = buf + m->run_off[q] + 4 * x;
-          const float* w = buf + m->run_off[q] + static_cast<long long>(n) * wq;
+          while (x >= (CW / 4) * m->run_nch[q]) x -= (CW / 4) * m->run_nch[q++];
+          i = x / (CW / 4);
+          col = x - i * (CW / 4);
+          const int n = m->run_n[q];
+          const int k0 = (sl * n) / slices, k1 = ((sl + 1) * n) / slices;
+          const float* rows = buf + m->run_off[q] + static_cast<long long>(i) * n * CW + 4 * col;
+          const float* w = buf + m->run_off[q] + static_cast<long long>(m->run_nch[q]) * n * CW + 4 * n;
 #pragma unroll 4
-          for (int k = sl; k < n; k += slices) {
+          for (int k = k0; k < k1; ++k) {
             const float wk = w[k];
-            if (wk != 0.f) {              // zero weight: an empty CTA's (unused) row
-              const float4 r = *reinterpret_cast<const float4*>(rows + static_cast<long long>(k) * wq);
-              acc.x += wk * r.x;
-              acc.y += wk * r.y;
-              acc.z += wk * r.z;
-              acc.w += wk * r.w;
-            }
+            const float4 r = *reinterpret_cast<const float4*>(rows + static_cast<long long>(k) * CW);
+            // a zero weight marks an empty CTA's row, never written: its bits are dropped
+            const bool z = wk == 0.f;
+            acc.x = fmaf(wk, z ? 0.f : r.x, acc.x);
+            acc.y = fmaf(wk, z ? 0.f : r.y, acc.y);
+            acc.z = fmaf(wk, z ? 0.f : r.z, acc.z);
+            acc.w = fmaf(wk, z ? 0.f : r.w, acc.w);
           }
         }
-        scratch[tid] = acc;
+        if (sl < slices) scratch[tid] = acc;
         __syncthreads();
-        if (sl == 0 && t < per && c4 < total_c4) {
-          float4 tot = scratch[tid];
+        if (act && sl == 0) {
+          float4 tot = acc;
           for (int j = 1; j < slices; ++j) {
-            const float4 v = scratch[tid + j];
+            const float4 v = scratch[j * per_c + t];
             tot.x += v.x;
             tot.y += v.y;
             tot.z += v.z;
             tot.w += v.w;
           }
-          int x = c4;
-          q = 0;
-          while (x >= (m->run_w[q] >> 2)) x -= m->run_w[q++] >> 2;
           const float inv = m->run_inv[q];
           const __nv_bfloat162 p0 = __floats2bfloat162_rn(tot.x * inv, tot.y * inv);
           const __nv_bfloat162 p1 = __floats2bfloat162_rn(tot.z * inv, tot.w * inv);
@@ -562,7 +596,7 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
           pk.x = *reinterpret_cast<const uint32_t*>(&p0);
           pk.y = *reinterpret_cast<const uint32_t*>(&p1);
           *reinterpret_cast<uint2*>(a.out + (static_cast<long long>(m->run_b[q]) * a.H + m->run_h[q]) *
-                                                a.d + m->run_d0[q] + 4 * x) = pk;
+                                                a.d + (m->run_c0[q] + i) * CW + 4 * col) = pk;
         }
         __syncthreads();
       }
@@ -632,7 +666,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&m->q_full, 1);
     mbar_init(&m->q_free, 1);
     mbar_init(&m->mma_done, 1);
+    mbar_init(&m->merge_bar, 1);
     m->abort = 0;
+    m->precut = 0;
     m->resc_tile = -1;
     fence_barrier_init();
   }
@@ -669,7 +705,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   int gtile_s = 0;       // S tiles issued / consumed
   int gtile_o = 0;       // PV tiles issued / P tiles produced
   const uint64_t evict_first = (warp == 0) ? l2_policy_evict_first() : 0ull;
-
   for (int batch = 0;; ++batch) {
     const int nseg = m->nseg;
     if (warp == 0 && a.k_new != nullptr) {
@@ -745,9 +780,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       __syncwarp();
       if (!m->more) {
-        // the producer's last loads are out: plan the fused merge meanwhile
+        // the producer's last loads are out: plan the fused merge and cut its first
+        // group of runs meanwhile
         for (int c = lane; c <= G; c += 32) m->ustart[c] = (c * U) / G;
         plan_merge(a, U, 0, m, lane);
+        __syncwarp();
+        if (lane == 0 && m->total_items > 0 && m->n_items > 0) {
+          m->cur_rec = 0;
+          m->cur_j = -1;
+          cut_group(a, m, LY::MISC_OFF / 4);
+          m->precut = 1;
+        }
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------- MMA issuer
@@ -974,9 +1017,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // a sequence held whole by this CTA is normalised and written out here; a split
         // one leaves its partial (O, m, l) in slot CTA + sequence for the merge
         const bool whole = sg.u0 == 0 && sg.u1 == seq_units(a, sg.b);
-        // the CTA's last segment: Q and the ring are idle, so the result is staged there
-        // and written with one bulk copy instead of per-thread scalar stores
+        // the CTA's last segment: Q and the ring are idle, so a whole sequence's output is
+        // staged there and written with bulk copies instead of per-thread scalar stores
         const bool staged = g == nseg - 1 && !m->more;
+        const long long S = static_cast<long long>(gridDim.x) + a.B;
         const long long slot = static_cast<long long>(blockIdx.x) + sg.b;
         if (t128 < a.H) {
           const int h = t128;
@@ -984,12 +1028,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (whole) {
             m->alpha[h] = 1.f / l;
           } else {
-            a.part_ml[(slot * a.H + h) * 2 + 0] = m_run;
-            a.part_ml[(slot * a.H + h) * 2 + 1] = l;
+            *reinterpret_cast<float4*>(a.part_ml + (h * S + slot) * 4) = make_float4(m_run, l, 0.f, 0.f);
           }
         }
         if (whole) named_bar_sync(1, 128);
-        float* po = a.part_o + slot * a.H * a.d;
         uint16_t* fo = a.out + static_cast<long long>(sg.b) * a.H * a.d;
         // staged: each 128-dim block is laid out [head][128] in its own region of the idle
         // ring / Q buffers; right after a block is complete, one thread per head stores
@@ -1003,6 +1045,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_ld_row<HP>(tmem + lane_addr + 2 * HP + db * HP, ob);
           tmem_wait_ld();
           const int col = db * 128 + row;       // this thread's head-dimension index
+          // the partial's rows: chunk db of head h in slot `slot` is 128 contiguous floats
+          float* po = a.part_o + (static_cast<long long>(db) * a.H * S + slot) * CW;
           if (staged) {
             const uint32_t base = smem_u32(smem) + db * blk_bytes + row * esz;
             if (whole) {
@@ -1017,18 +1061,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               for (int h = 0; h < HP; ++h)
                 if (h < a.H) st_shared_f32(base + h * 512u, ob[h]);
             }
-            fence_proxy_async_smem();
+            if (whole) fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (whole) {
               if (t128 < a.H) {
-                const uint8_t* src = smem + db * blk_bytes + t128 * 256;
+                const uint8_t* src = smem + db * blk_bytes + t128 * 256u;
                 bulk_store(fo + static_cast<long long>(t128) * a.d + db * 128, src, 256u);
                 issued = true;
               }
-            } else if (t128 == 0) {
-              // the partial's block db is [H][128] in both places: one copy
-              bulk_store(po + static_cast<long long>(db) * a.H * 128, smem + db * blk_bytes, blk_bytes);
-              issued = true;
+            } else {
+              // each warp copies whole 512-byte head rows: one 16-byte piece per lane
+              const float4* src = reinterpret_cast<const float4*>(smem + db * blk_bytes);
+              for (int h = sw; h < a.H; h += 4)
+                reinterpret_cast<float4*>(po + static_cast<long long>(h) * S * CW)[lane] = src[h * 32 + lane];
             }
           } else if (whole) {
 #pragma unroll
@@ -1038,10 +1083,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 fo[static_cast<long long>(h) * a.d + col] = *reinterpret_cast<const uint16_t*>(&v);
               }
           } else {
-            float* pb = po + static_cast<long long>(db) * a.H * 128 + row;
+            // for each head a warp writes 32 consecutive floats of the row (128 bytes)
 #pragma unroll
             for (int h = 0; h < HP; ++h)
-              if (h < a.H) pb[h * 128] = ob[h];
+              if (h < a.H) po[static_cast<long long>(h) * S * CW + row] = ob[h];
           }
         }
         if (issued) {
@@ -1100,10 +1145,10 @@ namespace {
 using lsa::attn::Args;
 
 // Workspace: the two grid-barrier counters on their own 256-byte line, then fp32
-// partial O [G+B][d/128][H][128] and partial (m, l) [G+B][H][2].
+// partial O [d/128][H][G+B][128] and partial (m, l, pad, pad) [H][G+B][4].
 size_t attn_ws_bytes(int B, int H, int d, int n_sm) {
   const size_t slots = static_cast<size_t>(n_sm) + static_cast<size_t>(B);
-  const size_t body = slots * static_cast<size_t>(H) * (static_cast<size_t>(d) + 2) * sizeof(float);
+  const size_t body = slots * static_cast<size_t>(H) * (static_cast<size_t>(d) + 4) * sizeof(float);
   return (body + 255) / 256 * 256 + 256;
 }
 

@@ -415,6 +415,9 @@ __device__ __forceinline__ long long ring_page(const StepArgs& a, int b, long lo
 // blocks oldest first, then the new tail page), and a zeroed tail page.
 __global__ void __launch_bounds__(THREADS) pass_setup_kernel(const StepArgs a, int p) {
   const int b = blockIdx.x, tid = threadIdx.x;
+  // the indexer launched next waits for this kernel's completion before it reads
+  // anything; letting it launch now overlaps its CTAs' set-up with this small kernel
+  grid_dependents_launch();
   const long long nb = static_cast<long long>(__ldg(a.nb0 + b)) + p;
   const long long first = nb - a.wb > 0 ? nb - a.wb : 0;
   if (tid == 0) {

@@ -28,6 +28,8 @@
 // counter only grows (by 2 x grid per launch), so no CTA has to reset it on the way out.
 #include "lsa_common.cuh"
 
+#include <atomic>
+
 namespace lsa {
 namespace idx {
 
@@ -213,7 +215,7 @@ __device__ __forceinline__ bool spin_until_geq64(const unsigned long long* count
     unsigned long long v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(counter) : "memory");
     if (v >= target) return true;
-    __nanosleep(32);
+    if (it >= 64) __nanosleep(32);   // the first polls back to back: barriers are short
     if (globaltimer_ns() - t0 > limit_ns || it > max_polls) return false;
   }
 }
@@ -560,6 +562,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) index_kernel(const Args a) {
     s->tab.resume_b = 0;
     s->tab.resume_base = 0;
   }
+  // Launched as a programmatic dependent: the set-up above overlaps the tail of the
+  // preceding kernel; nothing it may write is read before this point.
+  grid_dependency_wait();
+  grid_dependents_launch();
   __syncthreads();
   // ---- phase A. Warp 0 plans this CTA's keep words [W0, W1), and the KW copy warps
   // start the first chunk's K_idx copies at once; warps KW..: this CTA's rows of q.
@@ -768,12 +774,30 @@ lsa_status index_launch(const uint16_t* h, const uint16_t* w_q, const uint16_t* 
   cfg.blockDim = dim3(lsa::idx::NTHREADS);
   cfg.dynamicSmemBytes = kIndexSmem;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  // A programmatic dependent as well, so that the CTAs' set-up overlaps the preceding
+  // kernel's tail; a device that refuses the combination gets plain cooperative launches.
+  static std::atomic<int> pdl_state[64];   // 0 unknown/accepted, 1 refused (per device)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, lsa::idx::index_kernel, a) != cudaSuccess) {
+  const bool pdl = pdl_state[dev].load(std::memory_order_relaxed) == 0;
+  cfg.numAttrs = pdl ? 2 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, lsa::idx::index_kernel, a);
+  if (e == cudaErrorNotSupported && pdl) {
+    cudaGetLastError();
+    pdl_state[dev].store(1, std::memory_order_relaxed);
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, lsa::idx::index_kernel, a);
+  }
+  if (e != cudaSuccess) {
     cudaGetLastError();
     return LSA_ERR_CUDA;
   }

@@ -52,9 +52,9 @@ def test_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
-    # (n_sm + B) slots of H*(d + 2) floats, rounded to 256 bytes, + one 256-byte line of
+    # (n_sm + B) slots of H*(d + 4) floats, rounded to 256 bytes, + one 256-byte line of
     # grid-barrier counters
-    body = 149 * 64 * 514 * 4
+    body = 149 * 64 * 516 * 4
     assert lib.lsa_decode_attn_workspace_size(1, 64, 512, 148) == (body + 255) // 256 * 256 + 256
     assert lib.lsa_decode_attn_workspace_size(0, 64, 512, 148) == 0
     assert lib.lsa_index_workspace_size(1, 3, 128, 16256) > 3 * 128 * 4
