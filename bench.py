@@ -576,8 +576,10 @@ def e2e_measure(dec, wl, dev, passes, world, total_seqs=None):
     barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
+    t_host = time.perf_counter()
     for _ in range(passes):
         one_pass()
+    t_host = time.perf_counter() - t_host       # host time to enqueue every pass
     b.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), world)
@@ -589,7 +591,8 @@ def e2e_measure(dec, wl, dev, passes, world, total_seqs=None):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "copies_per_decode_step": {"h2d": 1, "d2h": 1},
             "copy_overlap": "copies on a second stream, double-buffered, ordered by events",
-            "ms_per_step": ms / passes, "api": "lsa_step (Python ctypes), pinned host buffers"}
+            "ms_per_step": ms / passes, "host_enqueue_ms_per_step": 1e3 * t_host / passes,
+            "api": "lsa_step (Python ctypes), pinned host buffers"}
 
 
 def delta_gather_report(wl, dev):

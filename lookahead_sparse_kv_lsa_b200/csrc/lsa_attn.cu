@@ -519,24 +519,38 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
         break;
       }
       // ---- split weights, one warp per run, from shared memory; an empty CTA's slot (no
-      // units, nothing written) gets weight 0
+      // units, nothing written; only possible when the grid has more CTAs than units)
+      // gets weight 0. Each lane loads its up to MAX_GRID / 32 slots at once.
       for (int q = warp; q < nr; q += NWARPS) {
         const int n = m->run_n[q];
         const float* ml = buf + m->run_off[q] + static_cast<long long>(m->run_nch[q]) * n * CW;
         float* w = const_cast<float*>(ml) + 4 * n;
         const long long c0 = m->run_clo[q];
+        constexpr int PER_LANE = MAX_GRID / 32;
+        float mk[PER_LANE], lk[PER_LANE];
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) {
+          const int k = lane + 32 * i;
+          mk[i] = -INFINITY;
+          lk[i] = 0.f;
+          if (k < n && (U >= G || m->ustart[c0 + k] != m->ustart[c0 + k + 1])) {
+            const float2 v = *reinterpret_cast<const float2*>(ml + 4 * k);
+            mk[i] = v.x;
+            lk[i] = v.y;
+          }
+        }
         float mx = -INFINITY;
-        for (int k = lane; k < n; k += 32)
-          if (m->ustart[c0 + k] != m->ustart[c0 + k + 1]) mx = fmaxf(mx, ml[4 * k]);
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) mx = fmaxf(mx, mk[i]);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float ls = 0.f;
-        for (int k = lane; k < n; k += 32) {
-          const bool live = m->ustart[c0 + k] != m->ustart[c0 + k + 1];
-          const float mk = ml[4 * k];
-          const float wk = (!live || mk == -INFINITY) ? 0.f : exp2f(mk - mx);
-          ls += wk == 0.f ? 0.f : wk * ml[4 * k + 1];
-          w[k] = wk;
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) {
+          const int k = lane + 32 * i;
+          const float wk = mk[i] == -INFINITY ? 0.f : exp2f(mk[i] - mx);
+          ls += wk == 0.f ? 0.f : wk * lk[i];
+          if (k < n) w[k] = wk;
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
@@ -566,17 +580,41 @@ __device__ __forceinline__ void merge_phase(const Args& a, Misc* m, float* buf, 
           const int k0 = (sl * n) / slices, k1 = ((sl + 1) * n) / slices;
           const float* rows = buf + m->run_off[q] + static_cast<long long>(i) * n * CW + 4 * col;
           const float* w = buf + m->run_off[q] + static_cast<long long>(m->run_nch[q]) * n * CW + 4 * n;
-#pragma unroll 4
-          for (int k = k0; k < k1; ++k) {
+          // a zero weight marks an empty CTA's row, never written: its bits are dropped.
+          // Rows go four at a time (loads first, two accumulators), joined in fixed order.
+          float4 acc2 = make_float4(0.f, 0.f, 0.f, 0.f);
+          int k = k0;
+          for (; k + 4 <= k1; k += 4) {
+            float wv[4];
+            float4 rv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              wv[e] = w[k + e];
+              rv[e] = *reinterpret_cast<const float4*>(rows + static_cast<long long>(k + e) * CW);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float4& A = (e & 1) ? acc2 : acc;
+              const bool z = wv[e] == 0.f;
+              A.x = fmaf(wv[e], z ? 0.f : rv[e].x, A.x);
+              A.y = fmaf(wv[e], z ? 0.f : rv[e].y, A.y);
+              A.z = fmaf(wv[e], z ? 0.f : rv[e].z, A.z);
+              A.w = fmaf(wv[e], z ? 0.f : rv[e].w, A.w);
+            }
+          }
+          for (; k < k1; ++k) {
             const float wk = w[k];
             const float4 r = *reinterpret_cast<const float4*>(rows + static_cast<long long>(k) * CW);
-            // a zero weight marks an empty CTA's row, never written: its bits are dropped
             const bool z = wk == 0.f;
             acc.x = fmaf(wk, z ? 0.f : r.x, acc.x);
             acc.y = fmaf(wk, z ? 0.f : r.y, acc.y);
             acc.z = fmaf(wk, z ? 0.f : r.z, acc.z);
             acc.w = fmaf(wk, z ? 0.f : r.w, acc.w);
           }
+          acc.x += acc2.x;
+          acc.y += acc2.y;
+          acc.z += acc2.z;
+          acc.w += acc2.w;
         }
         if (sl < slices) scratch[tid] = acc;
         __syncthreads();
@@ -752,10 +790,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               int ys[4];
 #pragma unroll
               for (int r = 0; r < 4; ++r) {
-                const int u = (tu0 + r < tu1) ? tu0 + r : tu0;  // pad with a valid unit
-                const int page = __ldg(bt + (u >> 1));
+                const int u = tu0 + r;
+                // rows past the tile's units: a box outside the map, zero-filled by the
+                // copy engine without reading memory (the softmax masks those rows)
+                const int page = u < tu1 ? __ldg(bt + (u >> 1)) : -1;
                 int y;
-                if (page < 0 || page >= a.n_pages) {
+                if (u >= tu1) {
+                  y = static_cast<int>(a.n_pages * 128);
+                } else if (page < 0 || page >= a.n_pages) {
                   set_err(a.err, LSA_DEVERR_BAD_PAGE);
                   y = static_cast<int>(a.n_pages * 128);  // outside the map: zero fill
                 } else {
