@@ -524,11 +524,12 @@ def e2e_measure(dec, wl, dev, passes, world, total_seqs=None):
     its inputs host->device in one copy (q, k_new and v_new packed in one pinned staging
     row; h joins step 0's row) and reads its output back device->host in one copy.
 
-    The copies run on a second stream and are ordered by events: step s's inputs go into
-    one of two device staging rows once step s-2 (the last reader of that row) is done,
-    the kernels of step s wait for their inputs, and step s's output is copied back from
-    one of two device output buffers once step s is done. So the copies overlap the
-    neighbouring steps' kernels, and every step still moves its own inputs and output."""
+    The copies run on two more streams, one per direction, ordered by events: step s's
+    inputs go into one of two device staging rows once step s-2 (the last reader of that
+    row) is done, the kernels of step s wait for their inputs, and step s's output is
+    copied back from one of two device output buffers once step s is done. So the copies
+    overlap the neighbouring steps' kernels, and every step still moves its own inputs
+    and output."""
     import torch
     import lookahead_sparse_kv_lsa_b200 as lsa
     c = wl.cfg
@@ -549,27 +550,32 @@ def e2e_measure(dec, wl, dev, passes, world, total_seqs=None):
               st[nq + nk:row].view(c.B, c.d), st[row:].view(c.L, c.B, c.D)) for st in stage]
     o_d = [torch.empty((c.B, c.H, c.d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     main = torch.cuda.current_stream()
-    copy = torch.cuda.Stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(c.tau)]
     ev_done = [torch.cuda.Event() for _ in range(c.tau)]
+    ev_out = [torch.cuda.Event() for _ in range(c.tau)]
 
     def one_pass():
         for s in range(c.tau):
             i = s & 1
             n = row + nh if s == 0 else row
-            with torch.cuda.stream(copy):
+            with torch.cuda.stream(up):
                 if s >= 2:
-                    copy.wait_event(ev_done[s - 2])          # staging row i is free again
+                    up.wait_event(ev_done[s - 2])            # staging row i is free again
                 stage[i][:n].copy_(host[s, :n], non_blocking=True)
-                ev_in[s].record(copy)
+                ev_in[s].record(up)
             main.wait_event(ev_in[s])
+            if s >= 2:
+                main.wait_event(ev_out[s - 2])               # output buffer i read back
             q_d, k_d, v_d, h_d = views[i]
             lsa.lsa_step(dec.state, s, h_d if s == 0 else None, q_d, k_d, v_d, o_d[i])
             ev_done[s].record(main)
-            with torch.cuda.stream(copy):
-                copy.wait_event(ev_done[s])
+            with torch.cuda.stream(down):
+                down.wait_event(ev_done[s])
                 out_host[s].copy_(o_d[i], non_blocking=True)
-        main.wait_stream(copy)
+                ev_out[s].record(down)
+        main.wait_stream(up)
+        main.wait_stream(down)
 
     one_pass()
     torch.cuda.synchronize()
@@ -590,7 +596,8 @@ def e2e_measure(dec, wl, dev, passes, world, total_seqs=None):
     return {"value": seqs * c.tau * passes / (ms * 1e-3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "copies_per_decode_step": {"h2d": 1, "d2h": 1},
-            "copy_overlap": "copies on a second stream, double-buffered, ordered by events",
+            "copy_overlap": "host->device and device->host copies on two more streams, "
+                            "double-buffered, ordered by events",
             "ms_per_step": ms / passes, "host_enqueue_ms_per_step": 1e3 * t_host / passes,
             "api": "lsa_step (Python ctypes), pinned host buffers"}
 
