@@ -556,6 +556,7 @@ def e2e_measure(dec, wl, dev, passes, world, total_seqs=None):
     ev_out = [torch.cuda.Event() for _ in range(c.tau)]
 
     def one_pass():
+        up.wait_stream(main)            # the previous pass's kernels are done with the rows
         for s in range(c.tau):
             i = s & 1
             n = row + nh if s == 0 else row
