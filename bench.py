@@ -260,15 +260,25 @@ def attn_bytes_per_step(cfg, ctx, n_sel, s):
     return total
 
 
-def index_launch_ms(dec, inp, reps=20, rounds=5):
+def index_launch_ms(dec, inp, reps=20, rounds=5, no_candidates=False):
     """Mean duration of one lsa_index launch: `reps` launches back to back in one CUDA
-    graph, replayed `rounds` times between two events (no event node between launches)."""
+    graph, replayed `rounds` times between two events (no event node between launches).
+    no_candidates: the same launch with every candidate count 0 (the projection, the two
+    grid barriers and the launch itself, with no keys to score: the structure's floor)."""
     import torch
+    import lookahead_sparse_kv_lsa_b200 as lsa
     stream = torch.cuda.Stream()
     g = torch.cuda.CUDAGraph()
+    zero = torch.zeros_like(dec.n_cand)
+    ids = torch.empty_like(dec.sel_ids)
+    cnt = torch.empty_like(dec.sel_cnt)
     with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
         for _ in range(reps):
-            dec.index(inp.h)
+            if no_candidates:
+                lsa.lsa_index(inp.h, dec.w_q, dec.bias, dec.k_idx, dec.kidx_off, zero,
+                              dec.max_cand, ids, cnt, dec.index_ws, dec.err)
+            else:
+                dec.index(inp.h)
     g.replay()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -829,6 +839,7 @@ def run_lsa(args, rank, world, local):
     ib = index_bytes(cfg, n_cand, n_sel)
     idx_in_pass = statistics.mean(idx_ms)
     idx_avg = index_launch_ms(dec, inp)
+    idx_floor = index_launch_ms(dec, inp, no_candidates=True)
     gather_bytes = sum(n_sel) * 2 * 64 * cfg.d * 2
     gth_avg = statistics.mean(gth_ms)
     h2d_peak = pinned_h2d_gbs(dev)
@@ -856,6 +867,7 @@ def run_lsa(args, rank, world, local):
                      "algorithmic_bytes_per_launch": attn_bytes,
                      "avg_launch_ms": attn_avg_ms},
         "indexer": {"ms": idx_avg, "timing": "20 launches back to back in one graph",
+                    "ms_no_candidates": idx_floor,
                     "ms_in_pass": idx_in_pass, "algorithmic_bytes": ib,
                     "achieved_GBs": ib / (idx_avg * 1e-3) / 1e9,
                     "frac": ib / (idx_avg * 1e-3) / 1e9 / hbm, "kept_blocks": n_sel,

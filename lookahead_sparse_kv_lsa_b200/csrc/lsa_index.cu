@@ -454,31 +454,39 @@ __device__ __forceinline__ void lowrank_rows(const Args& a, Smem* s, int k_lo, i
       const uint4* src = reinterpret_cast<const uint4*>(a.h + (static_cast<long long>(l) * a.B + b0) * a.D);
       for (int i = threadIdx.x; i < nb * g8; i += NTHREADS) hs[i] = __ldg(src + i);
       __syncthreads();
-      for (int k = row + warp; k < seg_hi; k += NWARPS) {
-        const uint4* wrow = reinterpret_cast<const uint4*>(a.w_1 + static_cast<long long>(k) * a.D);
-        float acc[LR_SEQ];
+      // two rows per warp at a time, all their 16-byte pieces requested before any use
+      for (int k = row + 2 * warp; k < seg_hi; k += 2 * NWARPS) {
+        const bool two = k + 1 < seg_hi;
+        const uint4* wrow0 = reinterpret_cast<const uint4*>(a.w_1 + static_cast<long long>(k) * a.D);
+        const uint4* wrow1 = reinterpret_cast<const uint4*>(a.w_1 + static_cast<long long>(two ? k + 1 : k) * a.D);
+        float acc0[LR_SEQ], acc1[LR_SEQ];
 #pragma unroll
-        for (int e = 0; e < LR_SEQ; ++e) acc[e] = 0.f;
+        for (int e = 0; e < LR_SEQ; ++e) acc0[e] = acc1[e] = 0.f;
         for (int g0 = 0; g0 < g8; g0 += 32 * LR_BATCH) {
-          uint4 w[LR_BATCH];
+          uint4 w0[LR_BATCH], w1[LR_BATCH];
 #pragma unroll
           for (int t = 0; t < LR_BATCH; ++t) {
             const int g = g0 + lane + 32 * t;
-            w[t] = g < g8 ? __ldg(wrow + g) : make_uint4(0u, 0u, 0u, 0u);
+            w0[t] = g < g8 ? __ldg(wrow0 + g) : make_uint4(0u, 0u, 0u, 0u);
+            w1[t] = (g < g8 && two) ? __ldg(wrow1 + g) : make_uint4(0u, 0u, 0u, 0u);
           }
 #pragma unroll
           for (int t = 0; t < LR_BATCH; ++t) {
             const int g = g0 + lane + 32 * t;
             if (g < g8) {
-              float wf[8];
-              unpack8(w[t], wf);
+              float wf0[8], wf1[8];
+              unpack8(w0[t], wf0);
+              unpack8(w1[t], wf1);
 #pragma unroll
               for (int e = 0; e < LR_SEQ; ++e) {
                 if (e < nb) {
                   float hf[8];
                   unpack8(hs[e * g8 + g], hf);
 #pragma unroll
-                  for (int i = 0; i < 8; ++i) acc[e] = fmaf(wf[i], hf[i], acc[e]);
+                  for (int i = 0; i < 8; ++i) {
+                    acc0[e] = fmaf(wf0[i], hf[i], acc0[e]);
+                    acc1[e] = fmaf(wf1[i], hf[i], acc1[e]);
+                  }
                 }
               }
             }
@@ -487,12 +495,20 @@ __device__ __forceinline__ void lowrank_rows(const Args& a, Smem* s, int k_lo, i
 #pragma unroll
         for (int e = 0; e < LR_SEQ; ++e) {
 #pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+          for (int o = 16; o >= 1; o >>= 1) {
+            acc0[e] += __shfl_xor_sync(0xffffffffu, acc0[e], o);
+            acc1[e] += __shfl_xor_sync(0xffffffffu, acc1[e], o);
+          }
         }
         if (lane == 0) {
 #pragma unroll
-          for (int e = 0; e < LR_SEQ; ++e)
-            if (e < nb) a.u[(static_cast<long long>(l) * a.B + b0 + e) * a.r + (k - l * a.r)] = acc[e];
+          for (int e = 0; e < LR_SEQ; ++e) {
+            if (e < nb) {
+              float* ub = a.u + (static_cast<long long>(l) * a.B + b0 + e) * a.r - static_cast<long long>(l) * a.r;
+              ub[k] = acc0[e];
+              if (two) ub[k + 1] = acc1[e];
+            }
+          }
         }
       }
     }
