@@ -409,8 +409,9 @@ lsa_status lsa_wait_selftest(const uint32_t* flag, uint32_t target, int64_t limi
  * 0 < top_p <= 1; any min_votes (<= 0 keeps every block, > n_layers none).
  * Ties in probability are ties in the fp32 logit, so the tie order is exact; where the
  * running mass meets top_p within rounding (fp32 probabilities, fp64 sums) the boundary
- * block may differ from an exact computation. Two launches on `stream`: one CTA per
- * (window, layer) for the sets, then one CTA per window for the vote.
+ * block may differ from an exact computation. Two launches on `stream`: persistent CTAs
+ * that take the (window, layer) rows in turn, then one CTA per window for the vote
+ * (a programmatic dependent launch where the device allows it).
  */
 #define LSA_DENOISE_MAX_BLOCKS 45056
 lsa_status lsa_denoise_labels(const float* logits, int32_t n_windows, int32_t n_layers,

@@ -118,7 +118,7 @@ def test_other_top_p(cuda_ok, p):
     check(x, run(x, p=p), p=p)
 
 
-@pytest.mark.parametrize("v", [-1, 0, 1, 2, 21, 22])
+@pytest.mark.parametrize("v", [-1, 0, 1, 2, 4, 8, 9, 21, 22])
 def test_vote_thresholds(cuda_ok, v):
     cfg = LI.DenoiseConfig(name="dn_v", windows=2, blocks=700, relevant=40, seed=5)
     x = LI.denoise_batch(cfg)
@@ -156,6 +156,40 @@ def test_edge_rows(cuda_ok):
     sets = bits(out["set_mask"], 1001)[0]
     assert sets[0][:601].all() and not sets[0][601:].any()
     assert near <= 1
+
+
+def test_edge_rows_bulk_copied(cuda_ok):
+    """The same rows over 8,192 blocks, a count the kernel copies in with bulk copies: the
+    all-equal and the narrow rows put more blocks in the boundary bin than the candidate
+    list holds, so they are split over the whole row first."""
+    N = 8192
+    x = _edge_rows(N).unsqueeze(0)
+    out = run(x, v=2)
+    near = check(x, out, v=2)
+    want = int(np.ceil(0.6 * N))                  # 4915.2 -> 4916 equal blocks, by id
+    assert out["set_cnt"][0][0] == want
+    sets = bits(out["set_mask"], N)[0]
+    assert sets[0][:want].all() and not sets[0][want:].any()
+    assert near <= 1
+
+
+def test_misaligned_logits(cuda_ok):
+    """Logits that start 4 bytes past a 16-byte boundary: the rows are read with plain
+    loads instead of bulk copies, with the same result."""
+    cfg = LI.DenoiseConfig(name="dn_m", windows=2, layers=5, blocks=4096, relevant=50, seed=21)
+    x = LI.denoise_batch(cfg)
+    W, L, N = x.shape
+    flat = torch.empty(W * L * N + 4, dtype=torch.float32)
+    flat[1:1 + W * L * N] = x.reshape(-1)
+    dev = torch.device("cuda")
+    big = flat.to(dev)
+    xv = big[1:1 + W * L * N].view(W, L, N)
+    assert xv.data_ptr() % 16 == 4
+    a = run(xv, v=1)
+    b = run(x, v=1)
+    for k in a:
+        np.testing.assert_array_equal(a[k], b[k])
+    check(x, a, v=1)
 
 
 def test_single_block_and_single_layer(cuda_ok):
