@@ -50,6 +50,7 @@ constexpr int DN_BINS = 16;           // first pass: whole logit units below the
 constexpr int DN_FINE = 256;          // splits of a bin or of a list
 constexpr int DN_RANK = 32;           // candidates ranked by one warp
 constexpr int DN_LIST = 2048;         // entries per list buffer
+constexpr int DN_INBIN = 4096;        // ids of the blocks of bin j0, listed when they fit
 constexpr int DN_MAX_REFINE = 8;      // 256-way key splits: 4 always suffice for 32-bit keys
 constexpr int DN_MAX_SPLIT = 12;      // 16-way row splits: 8 always suffice
 constexpr int DN_PLANES = 6;          // vote counter bit planes: counts up to 63 layers
@@ -80,7 +81,7 @@ struct DenoiseArgs {
 // pass's per-thread histogram columns and, after them, the two candidate list buffers
 // share the area `u`.
 struct __align__(16) Smem {
-  float u[DN_BINS * NT];     // hist columns | keys0, ids0, keys1, ids1 [DN_LIST each]
+  float u[DN_BINS * NT];     // hist columns | bin j0's ids [DN_INBIN] or keys1, ids1; keys0, ids0
   unsigned long long fmass[DN_FINE];  // split parts: mass in units of 2^-36
   uint32_t fcnt[DN_FINE];             // and block count
   double bsum[DN_BINS];
@@ -89,6 +90,8 @@ struct __align__(16) Smem {
   int32_t wcnt[NWARP];
   uint32_t wkmin[NWARP], wkmax[NWARP];
   int32_t cnt[2];            // entries appended to each list buffer
+  int32_t nin;               // blocks of bin j0 (their ids listed while they fit)
+  int32_t pad_;
   int32_t jsel;              // chosen bin or part (choose, choose_fine)
   int32_t csel;              // blocks in the chosen part (choose_fine)
   int32_t tau_id;            // mth_marked
@@ -100,12 +103,15 @@ struct __align__(16) Smem {
 
 extern __shared__ __align__(16) unsigned char dn_smem[];
 __device__ __forceinline__ Smem& sm() { return *reinterpret_cast<Smem*>(dn_smem); }
+// List buffer 0 takes the second half of u, buffer 1 the first half, which holds the ids
+// of bin j0's blocks until the candidates are listed.
 __device__ __forceinline__ uint32_t* list_k(int b) {
-  return reinterpret_cast<uint32_t*>(sm().u) + b * 2 * DN_LIST;
+  return reinterpret_cast<uint32_t*>(sm().u) + (1 - b) * 2 * DN_LIST;
 }
 __device__ __forceinline__ int32_t* list_i(int b) {
-  return reinterpret_cast<int32_t*>(sm().u) + b * 2 * DN_LIST + DN_LIST;
+  return reinterpret_cast<int32_t*>(sm().u) + (1 - b) * 2 * DN_LIST + DN_LIST;
 }
+__device__ __forceinline__ int32_t* inbin_ids() { return reinterpret_cast<int32_t*>(sm().u); }
 __device__ __forceinline__ float* row_x() { return reinterpret_cast<float*>(dn_smem + sizeof(Smem)); }
 __device__ __forceinline__ uint32_t* mask_words(int NW) {
   return reinterpret_cast<uint32_t*>(row_x() + static_cast<size_t>(NW) * 32);
@@ -272,7 +278,6 @@ __device__ __forceinline__ int block_scan(int v, int* total, uint32_t lo = 0xfff
   return before + incl - v;
 }
 
-__device__ __forceinline__ void choose_warp(double T, double acc, double top_p);
 __device__ __forceinline__ void choose_fine_warp(double T, double acc);
 
 // The answer of a choice over bins or parts: the chosen one, its block count (parts
@@ -286,17 +291,9 @@ struct Pick {
 
 // Scans 16 bins in s.bsum from the top for the first non-empty bin where acc + the
 // running mass reaches T (the last non-empty bin when rounding leaves the total short
-// of T). With top_p > 0, T is top_p times the bins' total. Warp 0 computes; every thread
-// has the answer after the barrier.
+// of T). With top_p > 0, T is top_p times the bins' total. Every warp computes the same
+// answer from 16 values, so no barrier follows; thread 0 also leaves it in s.
 __device__ __forceinline__ Pick choose(double T, double acc, double top_p = 0.0) {
-  Smem& s = sm();
-  if (threadIdx.x < 32) choose_warp(T, acc, top_p);
-  __syncthreads();
-  return Pick{s.jsel, s.csel, s.acc, s.T};
-}
-
-// choose() for the lanes of warp 0; lane 0 leaves the answer in s.
-__device__ __forceinline__ void choose_warp(double T, double acc, double top_p) {
   Smem& s = sm();
   const int lane = threadIdx.x & 31;
   const double bj = lane < DN_BINS ? s.bsum[lane] : 0.0;
@@ -312,13 +309,13 @@ __device__ __forceinline__ void choose_warp(double T, double acc, double top_p) 
   const uint32_t hit = __ballot_sync(0xffffffffu, bj > 0.0 && acc + incl >= T);
   const int j = hit ? __ffs(hit) - 1 : (nz ? 31 - __clz(nz) : 0);
   const double above = __shfl_sync(0xffffffffu, incl - bj, j);
-  if (lane == 0) {
+  if (threadIdx.x == 0) {
     s.jsel = j;
-    s.csel = 0;
     s.acc = acc + above;
     s.total_mass = total;
     s.T = T;
   }
+  return Pick{j, 0, acc + above, T};
 }
 
 // The same choice over the 256 split parts in s.fmass / s.fcnt (part 0 the largest
@@ -849,7 +846,10 @@ __global__ void __launch_bounds__(NT, 2) denoise_kernel(const __grid_constant__ 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) s.wmax[tid >> 5] = m;
-    if (tid == 0) s.cnt[0] = 0;  // this row's candidate list
+    if (tid == 0) {  // this row's lists
+      s.cnt[0] = 0;
+      s.nin = 0;
+    }
     if (tid < DN_FINE) {         // this row's split of bin j0
       s.fmass[tid] = 0ull;
       s.fcnt[tid] = 0u;
@@ -895,19 +895,52 @@ __global__ void __launch_bounds__(NT, 2) denoise_kernel(const __grid_constant__ 
     e.hi = last_bin ? INFINITY : e.lo + 1.0f;
     e.A = ref.R - e.lo;
     e.B = last_bin ? -INFINITY : e.A - 1.0f;
-    for (int q = tid; q < NW; q += NT) {
-      uint32_t up, gt;
-      if (exact) edge_word<true>(x4 + q * 8, rot, ref, e, up, gt);
-      else edge_word<false>(x4 + q * 8, rot, ref, e, up, gt);
+    // the loop runs the same rounds in every lane (warp-wide appends)
+    for (int q0 = 0; q0 < NW; q0 += NT) {
+      const int q = q0 + tid;
+      uint32_t up = 0u, gt = 0u;
+      if (q < NW) {
+        if (exact) edge_word<true>(x4 + q * 8, rot, ref, e, up, gt);
+        else edge_word<false>(x4 + q * 8, rot, ref, e, up, gt);
+      }
       const uint32_t in = gt & ~up;
-      mw[q] = up;
-      bw[q] = in;
-      for (uint32_t b = in; b != 0u; b &= b - 1u) {
-        const float v = x[q * 32 + __ffs(b) - 1];
-        fine_add(fine_part(ref, v, e.lo, last_bin), mass(v, ref.ml2));
+      if (q < NW) {
+        mw[q] = up;
+        bw[q] = in;
+      }
+      // bin j0's ids into the list: one shared atomic per warp
+      const int n = __popc(in);
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      int base = 0;
+      if (lane == 31 && total > 0) base = atomicAdd(&s.nin, total);
+      base = __shfl_sync(0xffffffffu, base, 31);
+      int pos = base + incl - n;
+      // bin j0's blocks into its 256-way split: the warp's listed blocks spread over its
+      // lanes; a warp whose blocks did not fit the list takes them word by word
+      if (base + total <= DN_INBIN) {
+        int32_t* ids = inbin_ids();
+        for (uint32_t b = in; b != 0u; b &= b - 1u) ids[pos++] = q * 32 + __ffs(b) - 1;
+        __syncwarp();
+        for (int j = lane; j < total; j += 32) {
+          const float v = x[ids[base + j]];
+          fine_add(fine_part(ref, v, e.lo, last_bin), mass(v, ref.ml2));
+        }
+      } else {
+        for (uint32_t b = in; b != 0u; b &= b - 1u) {
+          const float v = x[q * 32 + __ffs(b) - 1];
+          fine_add(fine_part(ref, v, e.lo, last_bin), mass(v, ref.ml2));
+        }
       }
     }
     __syncthreads();
+    const int nin = s.nin;
+    const bool listed = nin <= DN_INBIN;
     const Pick pf = choose_fine(T, acc);
     const int fsel = pf.j;
     const int c = pf.cnt;
@@ -918,22 +951,39 @@ __global__ void __launch_bounds__(NT, 2) denoise_kernel(const __grid_constant__ 
     {
       const bool list_it = c <= DN_LIST;
       uint32_t klo = 0xffffffffu, khi = 0u;
-      for (int q = tid; q < NW; q += NT) {
-        uint32_t up = 0u;
-        for (uint32_t b = bw[q]; b != 0u; b &= b - 1u) {
-          const int p = __ffs(b) - 1;
-          const float v = x[q * 32 + p];
+      if (listed) {
+        const int32_t* ids = inbin_ids();
+        for (int j = tid; j < nin; j += NT) {
+          const int id = ids[j];
+          const float v = x[id];
           const int f = fine_part(ref, v, e.lo, last_bin);
           if (f < fsel) {
-            up |= 1u << p;
+            mark(mw, NW, id, a.err);
           } else if (f == fsel) {
             const uint32_t key = order_key(v);
             klo = min(klo, key);
             khi = max(khi, key);
-            if (list_it) push(0, key, q * 32 + p);
+            if (list_it) push(0, key, id);
           }
         }
-        if (up != 0u) mw[q] |= up;
+      } else {
+        for (int q = tid; q < NW; q += NT) {
+          uint32_t up = 0u;
+          for (uint32_t b = bw[q]; b != 0u; b &= b - 1u) {
+            const int p = __ffs(b) - 1;
+            const float v = x[q * 32 + p];
+            const int f = fine_part(ref, v, e.lo, last_bin);
+            if (f < fsel) {
+              up |= 1u << p;
+            } else if (f == fsel) {
+              const uint32_t key = order_key(v);
+              klo = min(klo, key);
+              khi = max(khi, key);
+              if (list_it) push(0, key, q * 32 + p);
+            }
+          }
+          if (up != 0u) atomicOr(&mw[q], up);
+        }
       }
       int fixed = 0;
       if (list_it) {
@@ -990,12 +1040,42 @@ size_t smem_bytes(int32_t NW) {
 
 static_assert(sizeof(Smem) % 16 == 0, "the row starts 16-byte aligned");
 static_assert(4 * DN_LIST * 4 <= sizeof(float) * DN_BINS * NT, "both lists fit the shared area");
+static_assert(DN_INBIN <= 2 * DN_LIST, "bin j0's ids fit list buffer 1's place");
 static_assert(LSA_DENOISE_MAX_BLOCKS % 32 == 0, "whole mask words");
 static_assert(sizeof(Smem) + LSA_DENOISE_MAX_BLOCKS * 4 + LSA_DENOISE_MAX_BLOCKS / 4 <= 227 * 1024,
               "the longest row fits one CTA's shared memory");
 static_assert(LSA_DENOISE_MAX_BLOCKS * 4 < (1 << 20), "a row copy fits an mbarrier's count");
 static_assert(LSA_DENOISE_MAX_BLOCKS * 68719476736.0 < 9007199254740992.0,
               "a split part's fixed-point mass is exact in a double");
+
+// Launches kern<<<grid, NT, smem, st>>>(a) as a programmatic dependent of the stream's
+// preceding work, or plainly where the device refuses that (remembered per device).
+lsa_status launch_pdl(dim3 grid, size_t smem, cudaStream_t st,
+                      void (*kern)(const DenoiseArgs), const DenoiseArgs& a, int dev) {
+  static std::atomic<int> pdl_refused[64];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_refused[dev].load(std::memory_order_relaxed) ? 0 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
+  if (e == cudaErrorNotSupported && cfg.numAttrs == 1) {
+    cudaGetLastError();
+    pdl_refused[dev].store(1, std::memory_order_relaxed);
+    cfg.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+  }
+  return LSA_OK;
+}
 
 }  // namespace
 }  // namespace lsa
@@ -1051,32 +1131,12 @@ extern "C" lsa_status lsa_denoise_labels(const float* logits, int32_t n_windows,
     return LSA_ERR_CUDA;
   if (per_sm < 1) return LSA_ERR_CUDA;
   const int grid = static_cast<int>(std::min<int64_t>(a.rows, static_cast<int64_t>(per_sm) * sms));
+  // the vote as a programmatic dependent of the row kernel (measured: the row kernel
+  // itself is faster launched plainly, its CTAs then pair up on the SMs as they should)
+  if (dev < 0 || dev >= 64) return LSA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   denoise_kernel<<<grid, NT, smem, st>>>(a);
-  if (cudaPeekAtLastError() != cudaSuccess) return LSA_ERR_CUDA;
-  // the vote as a programmatic dependent (a device that refuses it gets a plain launch)
-  static std::atomic<int> pdl_refused[64];
-  if (dev < 0 || dev >= 64) return LSA_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_windows);
-  cfg.blockDim = dim3(NT);
-  cfg.dynamicSmemBytes = vote_smem_bytes(a.NW);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl_refused[dev].load(std::memory_order_relaxed) ? 0 : 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, vote_kernel, a);
-  if (e == cudaErrorNotSupported && cfg.numAttrs == 1) {
-    cudaGetLastError();
-    pdl_refused[dev].store(1, std::memory_order_relaxed);
-    cfg.numAttrs = 0;
-    e = cudaLaunchKernelEx(&cfg, vote_kernel, a);
-  }
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return LSA_ERR_CUDA;
-  }
-  return LSA_OK;
+  lsa_status r = cudaPeekAtLastError() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
+  if (r == LSA_OK) r = launch_pdl(dim3(n_windows), vote_smem_bytes(a.NW), st, vote_kernel, a, dev);
+  return r;
 }
