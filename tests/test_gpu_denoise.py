@@ -192,6 +192,21 @@ def test_misaligned_logits(cuda_ok):
     check(x, a, v=1)
 
 
+def test_large_magnitude_logits(cuda_ok):
+    """Rows whose maximum exceeds 2^22 in magnitude: the kernel bins by the rounded
+    difference to ceil(max) there instead of the exact one-add floor. At 3e7 the fp32
+    logits are multiples of 2, so most blocks tie with others."""
+    g = torch.Generator().manual_seed(77)
+    N = 4096
+    rows = [5.0e6 + torch.randn(N, generator=g) * 50.0,
+            -5.0e6 + torch.randn(N, generator=g) * 50.0,
+            3.0e7 + torch.randn(N, generator=g) * 1000.0,
+            4.0e6 + torch.randn(N, generator=g) * 3.0]
+    x = torch.stack(rows).to(torch.float32).unsqueeze(0)
+    out = run(x, v=2)
+    check(x, out, v=2)
+
+
 def test_single_block_and_single_layer(cuda_ok):
     x = torch.tensor([[[0.25]]])
     out = run(x, v=1)
