@@ -40,6 +40,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 
 namespace lsa {
 namespace {
@@ -1064,6 +1065,31 @@ static_assert(LSA_DENOISE_MAX_BLOCKS * 4 < (1 << 20), "a row copy fits an mbarri
 static_assert(LSA_DENOISE_MAX_BLOCKS * 68719476736.0 < 9007199254740992.0,
               "a split part's fixed-point mass is exact in a double");
 
+// Resident row-kernel CTAs per SM for `smem` bytes of dynamic shared memory on the current
+// device (the occupancy query, cached per device and size: it is host work per call
+// otherwise). 0 on error.
+int ctas_per_sm(size_t smem) {
+  struct Entry {
+    int dev;
+    size_t smem;
+    int per_sm;
+  };
+  static std::mutex mu;
+  static Entry done[64];
+  static int n_done = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].dev == dev && done[i].smem == smem) return done[i].per_sm;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, denoise_kernel, NT, smem) !=
+      cudaSuccess)
+    return 0;
+  if (n_done < 64) done[n_done++] = Entry{dev, smem, per_sm};
+  return per_sm;
+}
+
 // Launches kern<<<grid, NT, smem, st>>>(a) as a programmatic dependent of the stream's
 // preceding work, or plainly where the device refuses that (remembered per device).
 lsa_status launch_pdl(dim3 grid, size_t smem, cudaStream_t st,
@@ -1139,13 +1165,13 @@ extern "C" lsa_status lsa_denoise_labels(const float* logits, int32_t n_windows,
   a.err = err;
   // persistent: as many CTAs as fit at once, each taking every grid-th row
   const size_t smem = smem_bytes(a.NW);
-  int dev = 0, sms = 0, per_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, denoise_kernel, NT, smem) !=
-          cudaSuccess)
+  int dev = 0;
+  const int sms = lsa_host::sm_count();
+  const int per_sm = ctas_per_sm(smem);
+  if (cudaGetDevice(&dev) != cudaSuccess || sms < 1 || per_sm < 1) {
+    cudaGetLastError();
     return LSA_ERR_CUDA;
-  if (per_sm < 1) return LSA_ERR_CUDA;
+  }
   const int grid = static_cast<int>(std::min<int64_t>(a.rows, static_cast<int64_t>(per_sm) * sms));
   // the vote as a programmatic dependent of the row kernel (measured: the row kernel
   // itself is faster launched plainly, its CTAs then pair up on the SMs as they should)
